@@ -1,0 +1,374 @@
+#!/usr/bin/env python
+"""Benchmark of the CacheGen KV-cache codec (libcachegen) on B200.
+
+One step = one pass of the whole hot path over the Llama-2-7B-shaped MHA cache
+(32 layers x K/V x 32 kv_heads x 128 head_dim, fp16, 10,752 tokens = 7 chunks
+of 1,536; seeded AR(1) walks with 1% x8 outlier channels, seed 2; balanced
+level): cg_encode of all 7 chunks, then cg_decode_into of all 7 containers into
+one contiguous KV buffer.  Inputs (5.6 GB) are resident in HBM and larger than
+L2, so no flush is needed between iterations.
+
+Prints one JSON line.  `value` is the round-trip throughput (fp16 bytes per
+step / step time, GB/s); encode and decode are also reported on their own,
+with their fraction of the HBM roofline and the compression ratio.
+`--impl reference` times the plain CPU oracle instead (the only comparison
+arm this project has), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+WORKLOAD = dict(name="llama2_7b", L=32, H=32, D=128, T=10752, C=1536, seed=2, rho=0.95,
+                p_out=0.01, m_out=8.0, level=1)
+METRIC = "cg_decode / cg_encode GB/s (fp16 KV) on 1 B200, % of HBM roofline, compression ratio"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    try:
+        return json.loads((ROOT / "MEASURED_PEAKS.json").read_text())
+    except Exception:
+        return {}
+
+
+def _env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def _oracle_sample(threads: int):
+    """The CPU sample: one chunk of the workload cut into 16 independent 2-head
+    slices ([32, 2, 1536, 2, 128] each, 50 MB of fp16), round-tripped through the
+    oracle on up to `threads` host threads."""
+    import numpy as np
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    from kv_cache_compression_cachegen_b200 import synth
+    oracle.build()
+    w = WORKLOAD
+    slices = [synth.generate_cpu(w["L"], 2, w["D"], w["C"], seed=w["seed"] * 100 + i,
+                                 rho=w["rho"], p_out=w["p_out"], m_out=w["m_out"])
+              for i in range(16)]
+
+    def run_one(kv):
+        rc, cont = oracle.encode_chunk(kv, 0, w["C"], w["level"])
+        assert rc == 0
+        rc, vals, n, _ = oracle.decode_chunk(cont, w["L"], 2, w["D"], w["C"], w["level"])
+        assert rc == 0
+        return cont.size
+
+    nbytes = sum(s.nbytes for s in slices)
+    desc = (f"one {w['C']}-token chunk of the {w['name']} workload as 16 slices of "
+            f"[{w['L']},2,{w['C']},2,{w['D']}] fp16 ({nbytes / 1e6:.0f} MB), encode+decode")
+
+    def step():
+        t0 = time.perf_counter()
+        with ThreadPoolExecutor(threads) as ex:
+            sizes = list(ex.map(run_one, slices))
+        return time.perf_counter() - t0, sizes
+
+    return step, nbytes, desc
+
+
+def run_reference(args):
+    rank, world, _ = _env_rank()
+    if rank != 0:
+        return 0
+    threads = max(1, min(16, os.cpu_count() or 1))
+    step, nbytes, desc = _oracle_sample(threads)
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        dt, _ = step()
+        times.append(dt)
+    total = sum(times)
+    value = nbytes * args.steps / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8+f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD["name"], "sample": desc, "level": "balanced"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import kv_cache_compression_cachegen_b200 as cg
+    from kv_cache_compression_cachegen_b200 import synth
+    from kv_cache_compression_cachegen_b200 import torch_api as ta
+
+    rank, world, local = _env_rank()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cg.library()  # fails loudly if the native library is missing
+
+    w = WORKLOAD
+    L, H, D, T, C, level = w["L"], w["H"], w["D"], w["T"], w["C"], w["level"]
+    nch = -(-T // C)
+    shape = cg.Shape(L, H, D)
+    stream = torch.cuda.Stream(dev)
+    kv = torch.empty((L, 2, T, H, D), dtype=torch.int16, device=dev)
+    synth.generate_gpu(kv, L, H, D, T, w["seed"] + 1000 * rank, w["rho"], w["p_out"],
+                       w["m_out"], stream=stream)
+    enc = ta.Encoder(shape, C, nch, dev)
+    kv_out = torch.empty_like(kv)
+    status = ta.new_status(dev)
+    fp16_bytes = kv.numel() * 2
+
+    def encode():
+        cg.check(cg.cg_encode(shape, kv, T, 0, nch, C, level, None, enc.out, enc.stride,
+                              enc.sizes, enc.status, enc.workspace, enc.ws_bytes, stream))
+
+    def decode():
+        cg.check(cg.cg_decode_into(shape, enc.out, enc.stride, nch, C, level, kv_out, T, status,
+                                   stream))
+
+    torch.cuda.synchronize(dev)
+    for _ in range(max(args.warmup, 0)):
+        encode()
+        decode()
+    torch.cuda.synchronize(dev)
+    if ta.status_of(enc.status) != 0 or ta.status_of(status) != 0:
+        raise RuntimeError(f"codec status {ta.status_of(enc.status)} / {ta.status_of(status)}")
+    comp_bytes = int(enc.sizes.sum().item())
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        encode()
+        ev[i][1].record(stream)
+        decode()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    t_enc = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    t_dec = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    t_step = sum(t_enc) + sum(t_dec)
+    if world > 1:
+        tt = torch.tensor([t_step, sum(t_enc), sum(t_dec)], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step, te_sum, td_sum = tt.tolist()
+    else:
+        te_sum, td_sum = sum(t_enc), sum(t_dec)
+    ms_step = t_step / args.steps
+    ms_enc = te_sum / args.steps
+    ms_dec = td_sum / args.steps
+    peaks = _peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_HBM_GBS)
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    enc_gbps = fp16_bytes / ms_enc / 1e6
+    dec_gbps = fp16_bytes / ms_dec / 1e6
+    # algorithmic bytes: fp16 read + container write (encode); container read + fp16 write
+    alg = fp16_bytes + comp_bytes
+    enc_frac = alg / ms_enc / 1e6 / hbm
+    dec_frac = alg / ms_dec / 1e6 / hbm
+
+    # ---- end to end through the C ABI with host buffers --------------------
+    e2e = None
+    if not args.skip_e2e:
+        e2e = _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, C,
+                   level, T, fp16_bytes, world, dist)
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": round(fp16_bytes * world / ms_step / 1e6, 2),
+            "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u8+f32", "data": "synthetic",
+            "config": {"workload": f"{w['name']}: {L}x2x{H}x{D} fp16, {T} tokens = {nch} chunks "
+                                   f"of {C}, balanced, AR(1) rho {w['rho']} with "
+                                   f"{w['p_out']:.0%} x{w['m_out']:g} outliers, seed {w['seed']}",
+                       "step": "cg_encode(7 chunks) + cg_decode_into(7 chunks)",
+                       "l2": "inputs larger than L2 (5.6 GB), no flush",
+                       "parallelism": f"dp{world} (independent caches per GPU)"},
+            "encode_gbps": round(enc_gbps, 2), "decode_gbps": round(dec_gbps, 2),
+            "encode_ms": round(ms_enc, 4), "decode_ms": round(ms_dec, 4),
+            "encode_roofline_frac": round(enc_frac, 4), "decode_roofline_frac": round(dec_frac, 4),
+            "decode_frac_of_8tbs": round(alg / ms_dec / 1e6 / 8000.0, 4),
+            "encode_frac_of_8tbs": round(alg / ms_enc / 1e6 / 8000.0, 4),
+            "compression_ratio": round(fp16_bytes / comp_bytes, 4),
+            "container_bytes": comp_bytes,
+            "roofline": {"kernel": "decode_kernel (cg_decode_into)", "bound": "hbm",
+                         "achieved": round(alg / ms_dec / 1e6, 1), "peak": hbm,
+                         "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s",
+                         "frac": round(dec_frac, 4), "traffic": None,
+                         "algorithmic_bytes": alg},
+            "gpu_launches": 5 * args.steps,
+            "clocks": clocks,
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if not args.skip_cpu and world == 1:
+            line["cpu_baseline"] = _cpu_baseline()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, C, level, T,
+         fp16_bytes, world, dist):
+    """Host in, host out: pinned fp16 KV -> H2D -> cg_encode -> D2H containers (the
+    sender's side), then H2D containers -> cg_decode_into -> D2H status (the
+    receiver's side; the decoded KV stays in device memory, where the model reads it)."""
+    host_kv = torch.empty(kv.shape, dtype=kv.dtype, pin_memory=True)
+    host_kv.copy_(kv)
+    host_cont = torch.empty(enc.out.numel(), dtype=torch.uint8, pin_memory=True)
+    host_status = torch.empty(2, dtype=torch.int32, pin_memory=True)
+    sizes = enc.sizes.cpu().tolist()
+    dev_cont = torch.empty_like(enc.out)
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 3))
+    h2d = d2h = 0
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(steps):
+            kv.copy_(host_kv, non_blocking=True)
+            cg.check(cg.cg_encode(shape, kv, T, 0, nch, C, level, None, enc.out, enc.stride,
+                                  enc.sizes, enc.status, enc.workspace, enc.ws_bytes, stream))
+            for k in range(nch):  # each chunk's actual bytes leave the device
+                o = k * enc.stride
+                host_cont[o:o + sizes[k]].copy_(enc.out[o:o + sizes[k]], non_blocking=True)
+            for k in range(nch):
+                o = k * enc.stride
+                dev_cont[o:o + sizes[k]].copy_(host_cont[o:o + sizes[k]], non_blocking=True)
+            cg.check(cg.cg_decode_into(shape, dev_cont, enc.stride, nch, C, level, kv_out, T,
+                                       status, stream))
+            host_status[0:1].copy_(status, non_blocking=True)
+            host_status[1:2].copy_(enc.status, non_blocking=True)
+        t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if int(host_status[0]) != 0 or int(host_status[1]) != 0:
+        raise RuntimeError(f"e2e status {host_status.tolist()}")
+    ms = t0.elapsed_time(t1) / steps
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    comp = sum(sizes)
+    h2d = fp16_bytes + comp
+    d2h = comp + 8
+    return {"value": round(fp16_bytes * world / ms / 1e6, 3), "unit": "GB/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def _cpu_baseline():
+    threads = max(1, min(16, os.cpu_count() or 1))
+    step, nbytes, desc = _oracle_sample(threads)
+    dt, _ = step()
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle", "sample": desc}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,618 @@
+// encode.cu -- the CacheGen encoder: anchor range, anchor + delta quantiser
+// with per-head histograms and 12-bit table normalisation, rANS encoding of
+// one stream per (layer, K/V, token), the stream-offset prefix sum, and the
+// compaction of the streams into the container payload.
+//
+// [Practice] 1: quantise the difference to nearby tokens with a layer-wise
+// step, then entropy-code ("grouped entropy coding"); [Practice] 2.1: every
+// chunk is encoded on its own; [Practice] 3.1: the step tables; [Overview]
+// KV-cache quantisation mechanism: per-channel scale and zero point.
+//
+// Kernels, in launch order:
+//   quant_kernel    one CTA per (chunk, l, kv, h): anchor range -> zp, scale;
+//                   anchor codes and reconstructed anchors; delta symbols;
+//                   lane-replicated shared histogram; frequency table and the
+//                   encoder's per-symbol division constants.
+//   rans_kernel     one thread per stream (l, kv, t), symbols in reverse;
+//                   renormalisation words go through a per-thread ring in
+//                   shared memory and leave in 32-byte blocks, written
+//                   backwards into a per-stream scratch slot.
+//   scan_kernel     one CTA per chunk: exclusive prefix sum of stream lengths
+//                   -> offsets section, header, container size.
+//   compact_kernel  one warp per stream: scratch slot -> payload.
+#include <cuda_fp16.h>
+
+#include "cg_common.cuh"
+
+namespace cg {
+namespace {
+
+constexpr int kQThreads = 256;
+constexpr int kTileGroups = 16;
+constexpr int kTileTokens = kTileGroups * kGroup;  // 160
+constexpr int kRThreads = 128;                     // rANS streams per CTA
+constexpr int kRing = 64;                          // u16 ring entries per thread
+constexpr int kScanThreads = 1024;
+
+enum QuantMode { kModeEncode = 0, kModeTablesOnly = 1, kModeSuppliedTables = 2 };
+
+struct QSmem {
+  uint32_t hist;    // u32 [255][32]  lane-replicated counters (bank = lane)
+  uint32_t zp;      // f32 [256]
+  uint32_t sc;      // f32 [256]
+  uint32_t rcp;     // f32 [256]
+  uint32_t ahat;    // f32 [16][D + 4]
+  uint32_t red;     // f32 [2][512]   range reduction
+  uint32_t counts;  // u32 [256]
+  uint32_t total;
+};
+
+__host__ __device__ inline uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
+
+__host__ __device__ inline QSmem q_smem(int D) {
+  QSmem s;
+  s.hist = 0;
+  s.zp = a16(s.hist + 255u * 32u * 4u);
+  s.sc = s.zp + 1024u;
+  s.rcp = s.sc + 1024u;
+  s.ahat = s.rcp + 1024u;
+  s.red = a16(s.ahat + uint32_t(kTileGroups) * uint32_t(D + 4) * 4u);
+  s.counts = s.red + 2u * 512u * 4u;
+  s.total = a16(s.counts + 256u * 4u);
+  return s;
+}
+
+// Exact quantisation of d = x - a by a step s with precomputed r = RN(1/s):
+// y = RN(d * r) differs from RN(d / s) by under 2^-21 |y|, so when y is
+// further than that from every half-integer both round to the same integer.
+// The integer is read from the bits of yc + (1.5 * 2^23 + 127): the low byte
+// is u = q + 127.  `ok` turns false when the shortcut cannot decide (a value
+// near a half-integer, a huge |y|, or a non-finite input).
+__device__ __forceinline__ uint32_t quant_fast(float d, float r, bool& ok) {
+  const float y = __fmul_rn(d, r);
+  const float yc = fminf(fmaxf(y, -127.0f), 127.0f);
+  const float t = __fadd_rn(yc, 12583039.0f);
+  const float k = __fsub_rn(t, 12583039.0f);
+  const float e = __fsub_rn(yc, k);
+  const float gap = __fsub_rn(0.5f, fabsf(e));
+  const float m = __fmaf_rn(fabsf(y), -0x1p-21f, gap);  // exact sign of gap - |y| 2^-21
+  ok = ok && (m > 0.0f);
+  return __float_as_uint(t) & 0xFFu;
+}
+
+// The definition itself: u = clamp(roundf(RN(RN(x - a) / s)), -127, 127) + 127,
+// with s == 0 (a constant anchor channel) giving code 0.
+__device__ __forceinline__ uint32_t quant_exact(float x, float a, float s) {
+  if (s == 0.0f) return 127u;
+  const float y = __fdiv_rn(__fsub_rn(x, a), s);
+  const float r = fminf(fmaxf(roundf(y), -127.0f), 127.0f);
+  return uint32_t(int(r) + 127);
+}
+
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
+  return __reduce_add_sync(0xFFFFFFFFu, v);
+}
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+  return __reduce_max_sync(0xFFFFFFFFu, v);
+}
+
+// Normalise the 255 counts of one table to frequencies summing to 4096 (the
+// rule stated in cachegen.h).  One warp; lane holds u = 8 lane + i.  The
+// "decrement the largest" loop is applied level by level: all symbols tied at
+// the current maximum drop together to the next distinct value, and a final
+// partial round takes the tied symbols in increasing u order, which is what
+// the one-at-a-time rule does.
+__device__ void normalize_warp(const uint32_t* counts, uint64_t N, uint32_t f[8], int lane) {
+  uint32_t c[8];
+  uint32_t sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int u = lane * 8 + i;
+    c[i] = u < kAlphabet ? counts[u] : 0u;
+    uint32_t v = 0;
+    if (c[i]) {
+      v = uint32_t((uint64_t(c[i]) * kM) / N);
+      if (v < 1) v = 1;
+    }
+    f[i] = v;
+    sum += v;
+  }
+  sum = warp_sum_u32(sum);
+  if (sum < kM) {
+    // Largest count, ties to the smallest u: maximise (count, 255 - u).
+    unsigned long long key = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int u = lane * 8 + i;
+      if (c[i]) {
+        const unsigned long long k = (static_cast<unsigned long long>(c[i]) << 8) | uint32_t(255 - u);
+        key = k > key ? k : key;
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xFFFFFFFFu, key, o);
+      key = other > key ? other : key;
+    }
+    const int best = 255 - int(key & 0xFF);
+    if ((best >> 3) == lane) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (i == (best & 7)) f[i] += kM - sum;
+    }
+    return;
+  }
+  uint32_t excess = sum - kM;
+  while (excess > 0) {
+    uint32_t m1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (f[i] > 1 && f[i] > m1) m1 = f[i];
+    m1 = warp_max_u32(m1);
+    if (m1 == 0) break;  // unreachable: 255 ones sum to less than 4096
+    uint32_t tied = 0, m2 = 1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (f[i] == m1) ++tied;
+      else if (f[i] < m1 && f[i] > m2) m2 = f[i];
+    }
+    const uint32_t c1 = warp_sum_u32(tied);
+    m2 = warp_max_u32(m2);
+    if (uint64_t(c1) * (m1 - m2) <= excess) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (f[i] == m1) f[i] = m2;
+      excess -= c1 * (m1 - m2);
+    } else {
+      const uint32_t full = excess / c1, extra = excess % c1;
+      uint32_t rank = tied;  // exclusive prefix of tied counts over lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, rank, o);
+        if (lane >= o) rank += v;
+      }
+      rank -= tied;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (f[i] == m1) {
+          f[i] -= full + (rank < extra ? 1u : 0u);
+          ++rank;
+        }
+      }
+      excess = 0;
+    }
+  }
+}
+
+// Encoder constants of one symbol: x_max - 1, the Granlund-Montgomery
+// multiplier for exact 32-bit division by f ("Division by invariant integers
+// using multiplication", 1994, the N+1-bit case), cum, 4096 - f and the shifts.
+__device__ __forceinline__ uint4 enc_entry(uint32_t f, uint32_t cum) {
+  if (f == 0) return make_uint4(0xFFFFFFFFu, 0u, 0u, 0u);
+  const uint32_t lg = f == 1 ? 0u : 32u - __clz(f - 1);  // ceil(log2 f)
+  const uint32_t magic =
+      uint32_t(((1ull << 32) * ((1ull << lg) - f)) / f + 1ull);
+  const uint32_t sh1 = lg < 1 ? lg : 1u;
+  const uint32_t sh2 = lg > 0 ? lg - 1 : 0u;
+  return make_uint4((f << 20) - 1u, magic, cum | ((kM - f) << 16), sh1 | (sh2 << 8) | (f << 16));
+}
+
+__global__ void __launch_bounds__(kQThreads) quant_kernel(const EncParams p, const int mode) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int rest = blockIdx.x;
+  const int h = rest % p.H;
+  rest /= p.H;
+  const int kv = rest & 1;
+  rest >>= 1;
+  const int l = rest % p.L;
+  const int chunk = rest / p.L;
+  const int L = p.L, H = p.H, D = p.D, C = p.C;
+  const int64_t t0 = p.token_start + int64_t(chunk) * C;
+  const int n = int(min(int64_t(C), p.T - t0));
+  const int Gn = (n + kGroup - 1) / kGroup;
+  const int slab = l * 2 + kv;
+  const int tab = slab * H + h;
+  const uint64_t rs = uint64_t(H) * D;
+  const uint16_t* col = p.kv + (uint64_t(slab) * p.T + t0) * rs + uint64_t(h) * D;
+
+  const QSmem sm = q_smem(D);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + sm.hist);
+  float* zp = reinterpret_cast<float*>(smem + sm.zp);
+  float* sc = reinterpret_cast<float*>(smem + sm.sc);
+  float* rcp = reinterpret_cast<float*>(smem + sm.rcp);
+  float* ahat = reinterpret_cast<float*>(smem + sm.ahat);
+  float* red = reinterpret_cast<float*>(smem + sm.red);
+  uint32_t* counts = reinterpret_cast<uint32_t*>(smem + sm.counts);
+  const int astride = D + 4;
+
+  const Sections sec = sections(L, H, D, n);
+  uint8_t* cont = p.out ? p.out + uint64_t(chunk) * p.out_stride : nullptr;
+  // Table block offsets equal container offsets minus the header.
+  const uint64_t tb_zp = sec.zp - CG_HEADER_BYTES, tb_sc = sec.scale - CG_HEADER_BYTES,
+                 tb_fq = sec.freq - CG_HEADER_BYTES;
+  const bool want_hist = mode != kModeSuppliedTables;
+  const bool want_sym = mode != kModeTablesOnly;
+
+  if (want_hist)
+    for (int i = tid; i < kAlphabet * 32; i += kQThreads) hist[i] = 0;
+
+  // ---- Phase A: per-channel anchor range -> zp, scale (or the supplied ones).
+  bool nonfinite = false;
+  if (mode == kModeSuppliedTables) {
+    const uint8_t* tb = p.tables_in + uint64_t(chunk) * p.tables_stride;
+    for (int d = tid; d < D; d += kQThreads) {
+      zp[d] = reinterpret_cast<const float*>(tb + tb_zp)[uint64_t(tab) * D + d];
+      sc[d] = reinterpret_cast<const float*>(tb + tb_sc)[uint64_t(tab) * D + d];
+    }
+  } else {
+    const int np = D / 2;             // fp16 pairs per row
+    const int rp = kQThreads / np;    // anchor rows scanned in parallel (>= 2)
+    const int pi = tid % np, r = tid / np;
+    float lo0 = __int_as_float(0x7F800000), hi0 = -lo0, lo1 = lo0, hi1 = hi0;
+    if (r < rp) {
+      for (int g = r; g < Gn; g += rp) {
+        const uint32_t v =
+            __ldg(reinterpret_cast<const uint32_t*>(col + uint64_t(g) * kGroup * rs) + pi);
+        const float a = half_bits_to_float(uint16_t(v & 0xFFFF));
+        const float b = half_bits_to_float(uint16_t(v >> 16));
+        if (!isfinite(a) || !isfinite(b)) nonfinite = true;
+        lo0 = fminf(lo0, a);
+        hi0 = fmaxf(hi0, a);
+        lo1 = fminf(lo1, b);
+        hi1 = fmaxf(hi1, b);
+      }
+      red[r * D + 2 * pi] = lo0;
+      red[r * D + 2 * pi + 1] = lo1;
+      red[512 + r * D + 2 * pi] = hi0;
+      red[512 + r * D + 2 * pi + 1] = hi1;
+    }
+    __syncthreads();
+    for (int d = tid; d < D; d += kQThreads) {
+      float lo = red[d], hi = red[512 + d];
+      for (int j = 1; j < rp; ++j) {
+        lo = fminf(lo, red[j * D + d]);
+        hi = fmaxf(hi, red[512 + j * D + d]);
+      }
+      zp[d] = __fmul_rn(__fadd_rn(lo, hi), 0.5f);
+      sc[d] = __fdiv_rn(__fsub_rn(hi, lo), 254.0f);
+    }
+  }
+  __syncthreads();
+  for (int d = tid; d < D; d += kQThreads) {
+    rcp[d] = sc[d] == 0.0f ? 0.0f : __frcp_rn(sc[d]);
+    if (cont) {
+      reinterpret_cast<float*>(cont + sec.zp)[uint64_t(tab) * D + d] = zp[d];
+      reinterpret_cast<float*>(cont + sec.scale)[uint64_t(tab) * D + d] = sc[d];
+    }
+    if (p.tables_out) {
+      uint8_t* tb = p.tables_out + uint64_t(chunk) * p.tables_stride;
+      reinterpret_cast<float*>(tb + tb_zp)[uint64_t(tab) * D + d] = zp[d];
+      reinterpret_cast<float*>(tb + tb_sc)[uint64_t(tab) * D + d] = sc[d];
+    }
+  }
+  __syncthreads();
+
+  // ---- Phase B: quantise the chunk tile by tile (16 groups per tile).
+  const float step = step_of(p.level, l, L);
+  const float rstep = __frcp_rn(step);
+  const int nb = D / 16;            // 16-value blocks per row
+  const int tpw = 32 / nb;          // tokens per warp and pass
+  const int tw = lane / nb, b = lane % nb;
+  const bool lane_ok = lane < tpw * nb;
+  uint8_t* symc = p.sym + ((uint64_t(chunk) * L * 2 + slab) * H + h) * uint64_t(nb) * C * 16;
+
+  for (int tb = 0; tb < n; tb += kTileTokens) {
+    const int g0 = tb / kGroup;
+    const int ng = min(kTileGroups, Gn - g0);
+    // B1: anchor codes and reconstructed anchors of the tile's groups.
+    for (int idx = tid; idx < ng * D; idx += kQThreads) {
+      const int gi = idx / D, d = idx - gi * D;
+      const int t = tb + kGroup * gi;
+      const float x = half_bits_to_float(__ldg(col + uint64_t(t) * rs + d));
+      if (!isfinite(x)) nonfinite = true;
+      bool ok = true;
+      uint32_t u = quant_fast(__fsub_rn(x, zp[d]), rcp[d], ok);
+      if (!ok) u = quant_exact(x, zp[d], sc[d]);
+      const int c = int(u) - 127;
+      ahat[gi * astride + d] = __fadd_rn(zp[d], __fmul_rn(float(c), sc[d]));
+      if (want_hist) atomicAdd(&hist[u * 32 + lane], 1u);
+      if (want_sym) symc[(uint64_t(d >> 4) * C + t) * 16 + (d & 15)] = uint8_t(u);
+    }
+    __syncthreads();
+    // B2: the delta tokens of the tile; lane -> (token slot, 16-value block).
+    if (lane_ok) {
+      for (int k = warp * tpw + tw; k < ng * (kGroup - 1); k += (kQThreads / 32) * tpw) {
+        const int gi = k / (kGroup - 1);
+        const int t = tb + kGroup * gi + 1 + (k - gi * (kGroup - 1));
+        if (t >= n) continue;
+        const uint4* src = reinterpret_cast<const uint4*>(col + uint64_t(t) * rs + 16 * b);
+        const uint4 r0 = __ldg(src), r1 = __ldg(src + 1);
+        const uint32_t raw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+        const float4* ap = reinterpret_cast<const float4*>(ahat + gi * astride + 16 * b);
+        float a[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 v = ap[j];
+          a[4 * j] = v.x;
+          a[4 * j + 1] = v.y;
+          a[4 * j + 2] = v.z;
+          a[4 * j + 3] = v.w;
+        }
+        float x[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j]));
+          x[2 * j] = f2.x;
+          x[2 * j + 1] = f2.y;
+        }
+        bool ok = true;
+        uint32_t u[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) u[j] = quant_fast(__fsub_rn(x[j], a[j]), rstep, ok);
+        if (!ok) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (!isfinite(x[j])) nonfinite = true;
+            u[j] = quant_exact(x[j], a[j], step);
+          }
+        }
+        if (want_hist) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) atomicAdd(&hist[u[j] * 32 + lane], 1u);
+        }
+        if (want_sym) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            pk[j] = u[4 * j] | (u[4 * j + 1] << 8) | (u[4 * j + 2] << 16) | (u[4 * j + 3] << 24);
+          *reinterpret_cast<uint4*>(symc + (uint64_t(b) * C + t) * 16) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (nonfinite) set_status(p.status, CG_ERR_NONFINITE);
+
+  // ---- Phase C: histogram -> frequency table -> encoder constants.
+  if (want_hist) {
+    for (int u = tid; u < kAlphabet; u += kQThreads) {
+      uint32_t s = 0;
+      for (int j = 0; j < 32; ++j) s += hist[u * 32 + ((j + u) & 31)];
+      counts[u] = s;
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    uint32_t f[8];
+    if (mode == kModeSuppliedTables) {
+      const uint16_t* fq = reinterpret_cast<const uint16_t*>(
+          p.tables_in + uint64_t(chunk) * p.tables_stride + tb_fq) + uint64_t(tab) * 256;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = fq[lane * 8 + i];
+    } else {
+      normalize_warp(counts, uint64_t(n) * D, f, lane);
+    }
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pk[i] = f[2 * i] | (f[2 * i + 1] << 16);
+    const uint4 fv = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    if (cont)
+      reinterpret_cast<uint4*>(cont + sec.freq + uint64_t(tab) * 512)[lane] = fv;
+    if (p.tables_out)
+      reinterpret_cast<uint4*>(p.tables_out + uint64_t(chunk) * p.tables_stride + tb_fq +
+                               uint64_t(tab) * 512)[lane] = fv;
+    if (want_sym) {
+      uint32_t local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) local += f[i];
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      uint32_t cum = incl - local;
+      uint4* et = reinterpret_cast<uint4*>(p.etab) +
+                  ((uint64_t(chunk) * L * 2 + slab) * H + h) * 256;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        et[lane * 8 + i] = enc_entry(f[i], cum & 0xFFFF);
+        cum += f[i];
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t swap16(uint32_t v) { return __byte_perm(v, 0, 0x1032); }
+
+__global__ void __launch_bounds__(kRThreads, 4) rans_kernel(const EncParams p, const int check_f) {
+  __shared__ __align__(16) uint4 et[256];
+  __shared__ __align__(16) uint16_t ring[kRThreads * kRing];
+  const int tid = threadIdx.x;
+  const int C = p.C, L = p.L, H = p.H, D = p.D;
+  const int tiles = (C + kRThreads - 1) / kRThreads;
+  const int tile = blockIdx.x % tiles;
+  int rest = blockIdx.x / tiles;
+  const int slab = rest % (2 * L);
+  const int chunk = rest / (2 * L);
+  const int64_t t0 = p.token_start + int64_t(chunk) * C;
+  const int n = int(min(int64_t(C), p.T - t0));
+  if (tile * kRThreads >= n) return;
+  const int t = tile * kRThreads + tid;
+  const bool active = t < n;
+  const int nb = D / 16;
+  const uint64_t cs = uint64_t(chunk) * L * 2 + slab;
+  const uint4* etg = reinterpret_cast<const uint4*>(p.etab) + cs * H * 256;
+  const uint8_t* symc = p.sym + cs * H * uint64_t(nb) * C * 16;
+  const uint64_t ss = scratch_stride(H, D);
+  uint16_t* rend = reinterpret_cast<uint16_t*>(p.scratch + (cs * C + t + 1) * ss);
+  uint16_t* myring = ring + tid * kRing;
+
+  uint32_t x = kRansL, wp = 0, wf = 0;
+  bool bad = false;
+  for (int h = H - 1; h >= 0; --h) {
+    __syncthreads();
+    et[tid] = __ldg(etg + uint64_t(h) * 256 + tid);
+    et[tid + kRThreads] = __ldg(etg + uint64_t(h) * 256 + tid + kRThreads);
+    __syncthreads();
+    if (!active) continue;
+    for (int b = nb - 1; b >= 0; --b) {
+      const uint4 v =
+          __ldg(reinterpret_cast<const uint4*>(symc + ((uint64_t(h) * nb + b) * C + t) * 16));
+#pragma unroll
+      for (int k = 15; k >= 0; --k) {
+        const uint32_t word = (k >> 2) == 0 ? v.x : (k >> 2) == 1 ? v.y : (k >> 2) == 2 ? v.z : v.w;
+        const uint32_t u = (word >> (8 * (k & 3))) & 0xFFu;
+        const uint4 e = et[u];
+        if (x > e.x) {
+          myring[wp & (kRing - 1)] = uint16_t(x);
+          ++wp;
+          x >>= 16;
+        }
+        const uint32_t t1 = __umulhi(x, e.y);
+        const uint32_t q = (t1 + ((x - t1) >> (e.w & 0xFFu))) >> ((e.w >> 8) & 0xFFu);
+        x = x + (e.z & 0xFFFFu) + q * (e.z >> 16);
+        if (check_f) bad |= (e.w >> 16) == 0u;
+      }
+      if (wp - wf >= 16) {
+        const uint4* src = reinterpret_cast<const uint4*>(myring + (wf & (kRing - 1)));
+        const uint4 r0 = src[0], r1 = src[1];
+        uint4* dst = reinterpret_cast<uint4*>(rend - wf - 16);
+        dst[0] = make_uint4(swap16(r1.w), swap16(r1.z), swap16(r1.y), swap16(r1.x));
+        dst[1] = make_uint4(swap16(r0.w), swap16(r0.z), swap16(r0.y), swap16(r0.x));
+        wf += 16;
+      }
+    }
+  }
+  if (!active) return;
+  myring[wp & (kRing - 1)] = uint16_t(x);
+  ++wp;
+  myring[wp & (kRing - 1)] = uint16_t(x >> 16);
+  ++wp;
+  for (uint32_t k = wf; k < wp; ++k) rend[-1 - int64_t(k)] = myring[k & (kRing - 1)];
+  p.lens[cs * C + t] = wp;
+  if (bad) set_status(p.status, CG_ERR_MISMATCH);
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const EncParams p) {
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t s_total;
+  const int chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = p.C, L = p.L, H = p.H, D = p.D;
+  const int64_t t0 = p.token_start + int64_t(chunk) * C;
+  const int n = int(min(int64_t(C), p.T - t0));
+  const Sections sec = sections(L, H, D, n);
+  uint8_t* cont = p.out + uint64_t(chunk) * p.out_stride;
+  uint32_t* offs = reinterpret_cast<uint32_t*>(cont + sec.offsets);
+  const uint32_t* lens = p.lens + uint64_t(chunk) * L * 2 * C;
+  const int S = 2 * L * n;
+  const int per = (S + kScanThreads - 1) / kScanThreads;
+  const int s0 = min(S, tid * per), s1 = min(S, s0 + per);
+  uint32_t local = 0;
+  for (int s = s0; s < s1; ++s) local += lens[(s / n) * C + (s % n)];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t v = warp_tot[lane];
+    uint32_t wi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+      if (lane >= o) wi += u;
+    }
+    warp_tot[lane] = wi - v;
+    if (lane == 31) s_total = wi;
+  }
+  __syncthreads();
+  uint32_t run = warp_tot[warp] + incl - local;  // words before this thread's range
+  for (int s = s0; s < s1; ++s) {
+    offs[s] = 2u * run;
+    run += lens[(s / n) * C + (s % n)];
+  }
+  const uint64_t payload = 2ull * s_total;
+  if (tid == 0) {
+    offs[S] = uint32_t(payload);
+    const uint64_t total = up16(sec.payload + payload);
+    cg_header hd;
+    hd.magic = CG_MAGIC;
+    hd.version = CG_FORMAT_VERSION;
+    hd.level = uint8_t(p.level);
+    hd.group = uint8_t(kGroup);
+    hd.num_layers = uint32_t(L);
+    hd.num_kv_heads = uint32_t(H);
+    hd.head_dim = uint32_t(D);
+    hd.chunk_tokens = uint32_t(C);
+    hd.n_tokens = uint32_t(n);
+    hd.prob_bits = kProbBits;
+    hd.token_start = uint64_t(t0);
+    hd.payload_bytes = payload;
+    hd.total_bytes = total;
+    hd.reserved = 0;
+    const uint4* hs = reinterpret_cast<const uint4*>(&hd);
+    for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(cont)[i] = hs[i];
+    p.out_sizes[chunk] = total;
+    if (total > p.out_stride) set_status(p.status, CG_ERR_CAPACITY);
+  }
+  // Zero the padding after the offsets section and after the payload.
+  const uint64_t opad0 = sec.offsets + 4ull * (uint64_t(S) + 1);
+  if (tid < int(sec.payload - opad0)) cont[opad0 + tid] = 0;
+  const uint64_t total = up16(sec.payload + payload);
+  const uint64_t ppad0 = sec.payload + payload;
+  if (total <= p.out_stride && tid < int(total - ppad0)) cont[ppad0 + tid] = 0;
+}
+
+__global__ void __launch_bounds__(256) compact_kernel(const EncParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = p.C, L = p.L, H = p.H, D = p.D;
+  const uint64_t gs = uint64_t(blockIdx.x) * 8 + warp;
+  const uint64_t per_chunk = uint64_t(L) * 2 * C;
+  const int chunk = int(gs / per_chunk);
+  if (chunk >= p.num_chunks) return;
+  const uint64_t rem = gs - uint64_t(chunk) * per_chunk;
+  const int slab = int(rem / C), t = int(rem % C);
+  const int64_t t0 = p.token_start + int64_t(chunk) * C;
+  const int n = int(min(int64_t(C), p.T - t0));
+  if (t >= n) return;
+  const Sections sec = sections(L, H, D, n);
+  uint8_t* cont = p.out + uint64_t(chunk) * p.out_stride;
+  const uint32_t o0 = reinterpret_cast<const uint32_t*>(cont + sec.offsets)[uint64_t(slab) * n + t];
+  const uint64_t cs = uint64_t(chunk) * L * 2 + slab;
+  const uint32_t len = p.lens[cs * C + t];
+  if (sec.payload + o0 + 2ull * len > p.out_stride) return;  // capacity error already flagged
+  const uint16_t* src =
+      reinterpret_cast<const uint16_t*>(p.scratch + (cs * C + t + 1) * scratch_stride(H, D)) - len;
+  uint16_t* dst = reinterpret_cast<uint16_t*>(cont + sec.payload + o0);
+  for (uint32_t i = lane; i < len; i += 32) dst[i] = src[i];
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stream) {
+  const int mode =
+      build_only ? kModeTablesOnly : (p.tables_in ? kModeSuppliedTables : kModeEncode);
+  const QSmem sm = q_smem(p.D);
+  cudaError_t err = cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(sm.total));
+  if (err != cudaSuccess) return err;
+  const uint64_t qblocks = uint64_t(p.num_chunks) * p.L * 2 * p.H;
+  quant_kernel<<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, mode);
+  if ((err = cudaGetLastError()) != cudaSuccess || build_only) return err;
+  const uint64_t tiles = (p.C + kRThreads - 1) / kRThreads;
+  rans_kernel<<<unsigned(uint64_t(p.num_chunks) * p.L * 2 * tiles), kRThreads, 0, stream>>>(
+      p, mode == kModeSuppliedTables);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  scan_kernel<<<p.num_chunks, kScanThreads, 0, stream>>>(p);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const uint64_t streams = uint64_t(p.num_chunks) * p.L * 2 * p.C;
+  compact_kernel<<<unsigned((streams + 7) / 8), 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace cg

@@ -1,0 +1,69 @@
+"""Command-line round trip of the codec on one of the synthetic workloads.
+
+    python -m kv_cache_compression_cachegen_b200.roundtrip --workload mistral7b --level 1
+
+Generates the workload's KV cache on the GPU, then runs cg_encode of all its
+chunks followed by cg_decode_into of all containers, `--repeat` times, and
+prints the per-phase device times, the compression ratio and the status
+words.  Useful as a quick check of a build and as a small, fixed command for
+profilers.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+from . import Shape, cg_decode_into, cg_encode, check, library
+from . import synth
+from . import torch_api as ta
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="mistral7b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--level", type=int, default=1)
+    ap.add_argument("--chunk", type=int, default=0, help="chunk size (default: the workload's)")
+    ap.add_argument("--tokens", type=int, default=0, help="sequence length (default: workload's)")
+    ap.add_argument("--repeat", type=int, default=2)
+    args = ap.parse_args()
+    library()
+    w = synth.WORKLOADS[args.workload]
+    T = args.tokens or w.T
+    C = args.chunk or w.C
+    L, H, D = w.L, w.H, w.D
+    nch = -(-T // C)
+    dev = torch.device("cuda", 0)
+    kv = torch.empty((L, 2, T, H, D), dtype=torch.int16, device=dev)
+    synth.generate_gpu(kv, L, H, D, T, w.seed, w.rho, w.p_out, w.m_out)
+    shape = Shape(L, H, D)
+    enc = ta.Encoder(shape, C, nch, dev)
+    out = torch.empty_like(kv)
+    status = ta.new_status(dev)
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for _ in range(args.repeat):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        check(cg_encode(shape, kv, T, 0, nch, C, args.level, None, enc.out, enc.stride, enc.sizes,
+                        enc.status, enc.workspace, enc.ws_bytes, stream), "cg_encode")
+        e1.record(stream)
+        check(cg_decode_into(shape, enc.out, enc.stride, nch, C, args.level, out, T, status,
+                             stream), "cg_decode_into")
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append((e0.elapsed_time(e1), e1.elapsed_time(e2)))
+    comp = int(enc.sizes.sum().item())
+    res = {"workload": args.workload, "L": L, "H": H, "D": D, "T": T, "C": C, "chunks": nch,
+           "level": args.level, "fp16_bytes": kv.numel() * 2, "container_bytes": comp,
+           "ratio": round(kv.numel() * 2 / comp, 4),
+           "encode_ms": [round(a, 4) for a, _ in times],
+           "decode_ms": [round(b, 4) for _, b in times],
+           "encode_status": ta.status_of(enc.status), "decode_status": ta.status_of(status)}
+    print(json.dumps(res))
+    return 0 if res["encode_status"] == 0 and res["decode_status"] == 0 else 1
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())

@@ -1,0 +1,59 @@
+"""The native libraries build, load and export every declared entry point; the
+pure-host queries agree with the oracle.  No GPU is needed."""
+import ctypes
+import re
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def _declared(header: Path):
+    text = header.read_text(encoding="utf-8")
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cg_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = _declared(ROOT / "include" / "cachegen.h")
+    for need in ("cg_build_tables", "cg_encode", "cg_decode", "cg_decode_into"):
+        assert need in names
+
+
+def test_codec_library_exports_every_declared_symbol(native_built):
+    import kv_cache_compression_cachegen_b200 as cg
+    lib = ctypes.CDLL(str(cg.library_path()))
+    for header in (ROOT / "include").glob("*.h"):
+        for name in _declared(header):
+            assert hasattr(lib, name), name
+
+
+def test_synth_library_exports(native_built):
+    from kv_cache_compression_cachegen_b200 import synth
+    lib = ctypes.CDLL(str(synth._LIB))
+    assert hasattr(lib, "kvsynth_generate")
+
+
+@pytest.mark.parametrize("L,H,D,n", [(1, 1, 16, 10), (32, 8, 128, 1536), (32, 32, 128, 1536),
+                                     (48, 8, 128, 7), (4, 2, 64, 256)])
+def test_host_size_queries_match_oracle(native_built, oracle_lib, L, H, D, n):
+    import kv_cache_compression_cachegen_b200 as cg
+    assert cg.cg_section_offsets((L, H, D), n) == oracle_lib.sections(L, H, D, n)
+    assert cg.cg_encoded_bound((L, H, D), n) == oracle_lib.encoded_bound(L, H, D, n)
+    secs = oracle_lib.sections(L, H, D, 1)
+    assert cg.cg_tables_bytes((L, H, D)) == secs[2] + L * 2 * H * 512 - 64
+
+
+def test_argument_errors_are_synchronous(native_built):
+    import kv_cache_compression_cachegen_b200 as cg
+    shp = (4, 2, 64)
+    assert cg.library().cg_encoded_bound(ctypes.byref(cg.Shape(4, 2, 40)), 256,
+                                         ctypes.byref(ctypes.c_uint64())) == cg.CG_ERR_UNSUPPORTED
+    assert cg.cg_encode(shp, None, 256, 0, 1, 256, 1, None, None, 0, None, None, None, 0,
+                        stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_decode(shp, None, 64, 1, 256, 1, None, 0, None, stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_decode_into(shp, 16, 64, 1, 256, 5, 16, 256, 16, stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_build_tables(shp, 16, 256, 0, 2, 256, 1, 16, 16, stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_status_string(cg.CG_ERR_CORRUPT) == "corrupt container"
