@@ -233,6 +233,27 @@ cg_status cg_decode_into(const cg_shape* shape, const uint8_t* in_dev, uint64_t 
                          uint16_t* kv_dev, int64_t total_tokens, int32_t* status_dev,
                          cudaStream_t stream);
 
+/* cg_encode without caller-provided scratch.  The pages have no counterpart
+ * to this call; it exists for callers that cannot allocate device memory --
+ * an inference server that has reserved the whole GPU for its own pool, a
+ * plugin whose enqueue step must not call cudaMalloc, or a latency-critical
+ * path that cannot take an allocation's implicit synchronisation.  Arguments
+ * and results are those of cg_encode minus the workspace pair.  The scratch is
+ * one fixed 128 MiB block of device memory inside the library, reserved on
+ * every GPU that loads the library and held until the process exits; calls
+ * whose cg_encode_workspace_bytes exceeds 128 MiB return CG_ERR_CAPACITY.  The
+ * first call on a device looks up the block's device address (a host-side
+ * query); make that first call before any stream capture.  Every call uses
+ * the same block, so calls that overlap on the GPU (other streams, other
+ * host threads) race and must be serialised by the caller.  Nothing in the
+ * block needs clearing: each call writes every byte it reads.  No allocation
+ * of any kind happens in this call. */
+cg_status cg_encode_static(const cg_shape* shape, const uint16_t* kv_dev, int64_t total_tokens,
+                           int64_t token_start, int32_t num_chunks, int32_t chunk_tokens,
+                           cg_level level, const uint8_t* tables_dev, uint8_t* out_dev,
+                           uint64_t out_stride, uint64_t* out_sizes_dev, int32_t* status_dev,
+                           cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

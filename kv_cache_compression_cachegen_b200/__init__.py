@@ -18,7 +18,7 @@ __all__ = [
     "CG_ERR_NONFINITE", "CG_ERR_CUDA", "CG_ERR_UNSUPPORTED", "LEVELS", "CacheGenError",
     "Shape", "library", "library_path", "check", "cg_status_string", "cg_section_offsets",
     "cg_encoded_bound", "cg_tables_bytes", "cg_encode_workspace_bytes", "cg_build_tables",
-    "cg_encode", "cg_decode", "cg_decode_into",
+    "cg_encode", "cg_encode_static", "cg_decode", "cg_decode_into",
 ]
 
 CG_OK, CG_ERR_INVALID_ARG, CG_ERR_CAPACITY, CG_ERR_CORRUPT = 0, 1, 2, 3
@@ -68,6 +68,9 @@ _SIGNATURES = {
     "cg_encode": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_int64, ctypes.c_int64,
                                  ctypes.c_int32, ctypes.c_int32, ctypes.c_int, _P, _P,
                                  ctypes.c_uint64, _P, _P, _P, ctypes.c_uint64, _P]),
+    "cg_encode_static": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int, _P, _P, ctypes.c_uint64, _P, _P, _P]),
     "cg_decode": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_uint64, ctypes.c_int32,
                                  ctypes.c_int32, ctypes.c_int, _P, ctypes.c_uint64, _P, _P]),
     "cg_decode_into": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_uint64,
@@ -168,6 +171,17 @@ def cg_encode(shape, kv, total_tokens: int, token_start: int, num_chunks: int,
                                num_chunks, chunk_tokens, int(level), _ptr(tables), _ptr(out),
                                out_stride, _ptr(out_sizes), _ptr(status), _ptr(workspace),
                                workspace_bytes, _stream(stream))
+
+
+def cg_encode_static(shape, kv, total_tokens: int, token_start: int, num_chunks: int,
+                     chunk_tokens: int, level: int, tables, out, out_stride: int, out_sizes,
+                     status, stream=None) -> int:
+    """cg_encode with the library's own fixed scratch block (for callers that
+    cannot allocate device memory; see include/cachegen.h)."""
+    return library().cg_encode_static(ctypes.byref(_shape(shape)), _ptr(kv), total_tokens,
+                                      token_start, num_chunks, chunk_tokens, int(level),
+                                      _ptr(tables), _ptr(out), out_stride, _ptr(out_sizes),
+                                      _ptr(status), _stream(stream))
 
 
 def cg_decode(shape, inp, in_stride: int, num_chunks: int, chunk_tokens: int, level: int, out,
