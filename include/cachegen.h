@@ -60,15 +60,15 @@
  *                    u) is decremented by one
  *   cum[u] = sum of f[u'] for u' < u.
  *
- * rANS (32-bit state x, lower bound 2^16, 16-bit words, 12-bit probabilities):
- *   encode symbols j = H*D-1 down to 0 starting from x = 2^16:
- *       if x >= f << 20 (compared in 64 bits): emit x & 0xFFFF, x >>= 16
+ * rANS (32-bit state x in [2^15, 2^31), 16-bit words, 12-bit probabilities):
+ *   encode symbols j = H*D-1 down to 0 starting from x = 2^15:
+ *       if x >= f << 19: emit x & 0xFFFF, x >>= 16
  *       x = (x / f) * 4096 + x % f + cum
  *   then emit x & 0xFFFF and x >> 16.  The stream is the emitted words in
  *   reverse order, little-endian u16.  Decode reads x = (w0 << 16) | w1, then
  *   per symbol: slot = x & 4095, u = the symbol with cum[u] <= slot <
- *   cum[u] + f[u], x = f * (x >> 12) + slot - cum, and if x < 2^16 then
- *   x = (x << 16) | next word.  A valid stream ends with x == 2^16 and every
+ *   cum[u] + f[u], x = f * (x >> 12) + slot - cum, and if x < 2^15 then
+ *   x = (x << 16) | next word.  A valid stream ends with x == 2^15 and every
  *   word consumed.
  *
  * Container (one per chunk, little-endian, every section starts on a 16-byte

@@ -205,6 +205,7 @@ cg_status cg_encode(const cg_shape* shape, const uint16_t* kv_dev, int64_t total
   p.sym = w + ws.sym;
   p.etab = reinterpret_cast<uint32_t*>(w + ws.etab);
   p.lens = reinterpret_cast<uint32_t*>(w + ws.lens);
+  p.slabtot = reinterpret_cast<uint32_t*>(w + ws.slabtot);
   p.scratch = w + ws.scratch;
   p.status = status_dev;
   return from_cuda(cg::launch_encode(p, false, stream));

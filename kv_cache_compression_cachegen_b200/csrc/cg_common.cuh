@@ -16,7 +16,7 @@ namespace cg {
 constexpr int kGroup = CG_GROUP;          // tokens per anchor group
 constexpr uint32_t kProbBits = CG_PROB_BITS;
 constexpr uint32_t kM = 1u << kProbBits;  // every frequency table sums to 4096
-constexpr uint32_t kRansL = 1u << 16;     // lower bound of the 32-bit rANS state
+constexpr uint32_t kRansL = 1u << 15;     // lower bound of the 32-bit rANS state (x < 2^31)
 constexpr int kAlphabet = 255;            // symbols u = v + 127 for v in [-127, 127]
 
 // Limits of this implementation (checked by the C ABI before any launch).
@@ -87,6 +87,7 @@ struct EncWorkspace {
   uint64_t sym;      // u8  [chunks][L][2][H][D/16][C][16]
   uint64_t etab;     // u32 [chunks][L][2][H][256][4]
   uint64_t lens;     // u32 [chunks][L][2][C]
+  uint64_t slabtot;  // u32 [chunks][L][2]   words of each (layer, K/V)'s streams
   uint64_t scratch;  // u8  [chunks][L][2][C][scratch_stride]
   uint64_t total;
 };
@@ -99,7 +100,8 @@ __host__ __device__ inline EncWorkspace enc_workspace(int L, int H, int D, int C
   w.sym = 0;
   w.etab = up256(w.sym + streams * uint64_t(H) * D);
   w.lens = up256(w.etab + uint64_t(chunks) * L * 2 * H * 256 * 16);
-  w.scratch = up256(w.lens + streams * 4);
+  w.slabtot = up256(w.lens + streams * 4);
+  w.scratch = up256(w.slabtot + uint64_t(chunks) * L * 2 * 4);
   w.total = up256(w.scratch + streams * scratch_stride(H, D));
   return w;
 }
@@ -122,6 +124,7 @@ struct EncParams {
   uint8_t* sym;            // workspace sections
   uint32_t* etab;
   uint32_t* lens;
+  uint32_t* slabtot;
   uint8_t* scratch;
   int32_t* status;
 };

@@ -14,16 +14,24 @@
 // frequency table, so the CTA walks the heads in lockstep:
 //   iteration it:  anchor warp decodes head it      with table it % 3,
 //                  delta warps decode head it - 1   with table (it-1) % 3,
-//                  all threads build the slot table of head it + 1.
+//                  all threads fill the slot table of head it + 1,
+//                  one warp scans the frequencies of head it + 2.
 // The anchor warp runs one head ahead so that the reconstructed anchors a_g of
 // head it-1 (fp32, in shared memory) are ready when the delta warps need them;
 // one __syncthreads per head separates the iterations.
 //
-// Per symbol a thread does one shared-memory slot lookup, the rANS state
-// update, an optional 16-bit refill from its own stream (L1-cached global
-// loads), and the dequantisation a + (float)q * s with IEEE round-to-nearest
-// adds and multiplies (no contraction).  (float)q * step is exact-rounded once,
-// so it is read from a 255-entry table of the layer's products.
+// Compressed words reach a thread through a 64-byte ring in shared memory
+// (four 16-byte blocks).  Every 8 symbols the thread issues at most one
+// cp.async for the next block of its stream and waits only for the blocks
+// issued two steps earlier; since 8 symbols consume at most 8 words (one
+// block), the words a step can read were always requested at least two steps
+// before, so global-memory latency stays off the decode chain.
+//
+// Per symbol: one slot-table lookup, the state update, an optional 16-bit
+// refill from the ring, and the dequantisation a + (float)q * s with IEEE
+// round-to-nearest adds and multiplies (no contraction).  The slot entry keeps
+// the symbol in its top byte, so (float)q comes from a byte permute and one
+// exact subtraction instead of a second shared-memory lookup.
 #include <cuda_fp16.h>
 
 #include "cg_common.cuh"
@@ -36,15 +44,20 @@ constexpr int kDeltaPerGroup = kGroup - 1;             // 9
 constexpr int kWarps = 1 + kDeltaPerGroup;             // anchor warp + 9 delta warps
 constexpr int kThreads = 32 * kWarps;                  // 320
 constexpr int kUnitTokens = kUnitGroups * kGroup;      // 320
-constexpr int kCumStride = 258;                        // u16 per head: cum[0..256] + pad
+constexpr uint32_t kCumBuf = 800;                      // bytes per compacted-table buffer
+constexpr uint32_t kRingBytes = 64;                    // per thread: 4 blocks of 16 bytes
+constexpr uint32_t kRingBlocks = kRingBytes / 16;
+constexpr uint32_t kRingWords = kRingBytes / 2;
 
 // Dynamic shared memory layout (byte offsets), a function of H and D.
 struct DecSmem {
-  uint32_t tbl;     // u32 [3][4096]   slot tables, packed (f << 20) | (u << 12) | (slot - cum)
+  uint32_t tbl;     // u32 [3][4096]  slot tables, packed (u << 24) | (f << 12) | (slot - cum)
   uint32_t ahat;    // f32 [2][32][D + 4]  reconstructed anchors of the last two heads
-  uint32_t cum;     // u16 [H][258]    cumulative frequencies of every head
-  uint32_t lut;     // f32 [256]       (float)(u - 127) * step for this layer
-  uint32_t single;  // i32 [H]         symbol of a one-symbol table, else -1
+  uint32_t ring;    // u8  [320][64]  per-thread word rings (64-byte aligned)
+  uint32_t cum;     // [2] x {u16 pcum[257], u8 psym[256], i32 nz}: the next two heads' present
+                    //        symbols in order and their cumulative frequencies
+  uint32_t zs;      // f32 [2][2][D]  zero points and scales of the anchor warp's next heads
+  uint32_t single;  // i32 [H]        symbol of a one-symbol table, else -1
   uint32_t total;
 };
 
@@ -54,52 +67,177 @@ __host__ __device__ inline DecSmem dec_smem(int H, int D) {
   DecSmem s;
   s.tbl = 0;
   s.ahat = al16(s.tbl + 3u * 4096u * 4u);
-  s.cum = al16(s.ahat + 2u * kUnitGroups * uint32_t(D + 4) * 4u);
-  s.lut = al16(s.cum + uint32_t(H) * kCumStride * 2u);
-  s.single = al16(s.lut + 256u * 4u);
+  // the rings are realigned to 64 bytes in the absolute shared address space,
+  // hence the 64 bytes of slack
+  s.ring = al16(s.ahat + 2u * kUnitGroups * uint32_t(D + 4) * 4u);
+  s.cum = al16(s.ring + uint32_t(kThreads) * kRingBytes + 64u);
+  s.zs = al16(s.cum + 2u * kCumBuf);
+  s.single = al16(s.zs + 4u * uint32_t(D) * 4u);
   s.total = al16(s.single + uint32_t(H) * 4u);
   return s;
 }
 
-__device__ __forceinline__ uint16_t ldg_u16(const uint16_t* p) { return __ldg(p); }
+// ---- stream ring ------------------------------------------------------------
+// Word q of the stream (absolute u16 index in the container) lives at ring byte
+// offset 2 * (q mod 32): block b = q / 8 occupies slot b mod 4.
+struct Ring {
+  const uint8_t* gbase;  // container start (16-byte aligned)
+  uint32_t rb;           // shared-memory address of this thread's ring (64-byte aligned)
+  uint32_t fb;           // next 16-byte block of the container to request
+  uint32_t lim;          // number of 16-byte blocks in the container
+};
 
-// Fill the 4096-entry slot table of one head: thread tid covers slots
-// [tid*4096/kThreads, (tid+1)*4096/kThreads).  The symbol of the first slot is
-// found by binary search over the cumulative frequencies; the rest by walking.
-__device__ __forceinline__ void fill_table(uint32_t* tbl, const uint16_t* cum, int tid) {
-  const int s0 = (tid * int(kM)) / kThreads;
-  const int s1 = ((tid + 1) * int(kM)) / kThreads;
-  int lo = 0, hi = kAlphabet;  // cum[lo] <= s0 < cum[hi]; cum[255] == 4096
+// Request the next block if the ring has room (predicated, no branch), then
+// close the group.
+__device__ __forceinline__ void ring_issue(Ring& r, uint32_t p) {
+  const uint32_t want = min((p >> 3) + kRingBlocks, r.lim);
+  const uint32_t dst = r.rb + (r.fb & (kRingBlocks - 1)) * 16u;
+  const uint8_t* src = r.gbase + uint64_t(r.fb) * 16u;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      "setp.lt.u32 p, %0, %1;\n\t"
+      "@p cp.async.cg.shared.global [%2], [%3], 16;\n\t"
+      "@p add.u32 %0, %0, 1;\n\t"
+      "cp.async.commit_group;\n\t"
+      "}\n"
+      : "+r"(r.fb)
+      : "r"(want), "r"(dst), "l"(src)
+      : "memory");
+}
+
+__device__ __forceinline__ void ring_wait_two_steps() {
+  asm volatile("cp.async.wait_group 2;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void ring_wait_all() {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];\n" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ring_addr(const Ring& r, uint32_t q) {
+  return r.rb + ((q & (kRingWords - 1)) << 1);
+}
+
+// Compacted table of one head: the present symbols in increasing order
+// (psym), their cumulative frequencies (pcum, with pcum[nz] = 4096) and nz.
+struct CumBuf {
+  uint16_t* pcum;
+  uint8_t* psym;
+  int* nz;
+};
+
+__device__ __forceinline__ CumBuf cum_buf(uint8_t* base) {
+  return CumBuf{reinterpret_cast<uint16_t*>(base), base + 520, reinterpret_cast<int*>(base + 784)};
+}
+
+// One warp turns a head's 256 frequencies (already in registers: lane holds
+// symbols 8 lane .. 8 lane + 7) into its compacted table.
+__device__ __forceinline__ void cum_compact(const uint4 raw, CumBuf cb, int lane) {
+  const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t f[8];
+  uint32_t local = 0, present = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = wv[i] & 0xFFFF;
+    f[2 * i + 1] = wv[i] >> 16;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    local += f[i];
+    present += f[i] != 0;
+  }
+  uint32_t incl = local, pincl = present;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    const uint32_t pv = __shfl_up_sync(0xFFFFFFFFu, pincl, o);
+    if (lane >= o) {
+      incl += v;
+      pincl += pv;
+    }
+  }
+  uint32_t run = incl - local, at = pincl - present;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (f[i] != 0) {
+      cb.pcum[at] = uint16_t(run);
+      cb.psym[at] = uint8_t(lane * 8 + i);
+      ++at;
+    }
+    run += f[i];
+  }
+  if (lane == 31) {
+    cb.pcum[pincl] = uint16_t(kM);
+    *cb.nz = int(pincl);
+  }
+}
+
+// Fill the 4096-entry slot table of one head: threads 0..255 each write 16
+// consecutive slots with four 16-byte stores.  The symbol of the first slot is
+// found by binary search over the present symbols' cumulative frequencies;
+// each later slot advances at most one present symbol.
+__device__ __forceinline__ void fill_table(uint32_t* tbl, CumBuf cb, int tid) {
+  if (tid >= 256) return;
+  const int s0 = tid * 16;
+  int lo = 0, hi = *cb.nz;  // pcum[lo] <= s0 < pcum[hi]; pcum[nz] == 4096
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (int(cum[mid]) <= s0) lo = mid; else hi = mid;
+    if (int(cb.pcum[mid]) <= s0) lo = mid; else hi = mid;
   }
-  int u = lo;
-  int cc = cum[u], cn = cum[u + 1];
-  for (int s = s0; s < s1; ++s) {
-    while (cn <= s) {
-      ++u;
-      cc = cn;
-      cn = cum[u + 1];
+  int i = lo;
+  int cc = cb.pcum[i], cn = cb.pcum[i + 1];
+  uint32_t u = cb.psym[i];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t ent[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int s = s0 + 4 * q + k;
+      if (cn <= s) {  // one step reaches the next present symbol
+        ++i;
+        cc = cn;
+        cn = cb.pcum[i + 1];
+        u = cb.psym[i];
+      }
+      ent[k] = (u << 24) | (uint32_t(cn - cc) << 12) | uint32_t(s - cc);
     }
-    tbl[s] = (uint32_t(cn - cc) << 20) | (uint32_t(u) << 12) | uint32_t(s - cc);
+    *reinterpret_cast<uint4*>(tbl + s0 + 4 * q) = make_uint4(ent[0], ent[1], ent[2], ent[3]);
   }
 }
 
 // One rANS decode step: returns the packed table entry of the decoded symbol.
-template <bool kClamp>
-__device__ __forceinline__ uint32_t rans_step(uint32_t& x, uint64_t& p, uint32_t& w,
-                                              const uint32_t* __restrict__ tbl,
-                                              const uint16_t* __restrict__ w16, uint64_t limit) {
+// The refill is predicated, not branched: x = (x << 16) | w, advance the ring
+// address ra (wrapping inside the thread's 64 bytes) and load the next word.
+__device__ __forceinline__ uint32_t rans_step(uint32_t& x, uint32_t& ra, uint32_t& w,
+                                              const uint32_t* __restrict__ tbl, uint32_t rb) {
   const uint32_t e = tbl[x & (kM - 1)];
-  x = (e >> 20) * (x >> kProbBits) + (e & (kM - 1));
-  if (x < kRansL) {
-    x = (x << 16) | w;
-    ++p;
-    const uint64_t q = kClamp ? (p < limit ? p : limit - 1) : p;
-    w = ldg_u16(w16 + q);
-  }
+  x = ((e >> 12) & (kM - 1)) * (x >> kProbBits) + (e & (kM - 1));
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      ".reg .u32 t;\n\t"
+      "setp.lt.u32 p, %0, %4;\n\t"
+      "@p prmt.b32 %0, %2, %0, 0x5410;\n\t"
+      "@p add.u32 t, %1, 2;\n\t"
+      "@p and.b32 t, t, 63;\n\t"
+      "@p or.b32 %1, t, %3;\n\t"
+      "@p ld.shared.u16 %2, [%1];\n\t"
+      "}\n"
+      : "+r"(x), "+r"(ra), "+r"(w)
+      : "r"(rb), "n"(kRansL));
   return e;
+}
+
+// (float)(u - 127) for the symbol u in the entry's top byte: the bits
+// 0x4B0000uu are the float 2^23 + u, and subtracting 2^23 + 127 is exact.
+__device__ __forceinline__ float sym_value(uint32_t e) {
+  return __fsub_rn(__uint_as_float(__byte_perm(e, 0x4B000000u, 0x7653)), 8388735.0f);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -107,56 +245,63 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Delta lane: decode head h of its stream into 8-value blocks.
-template <bool kClamp>
-__device__ __forceinline__ void decode_delta_head(uint32_t& x, uint64_t& p, uint32_t& w,
-                                                  const uint32_t* __restrict__ tbl,
-                                                  const float* __restrict__ lut,
+// Stream position of a thread: p (absolute word index of the next unread
+// word, kept per step) and ra (its ring address, advanced per refill).
+struct Pos {
+  uint32_t p, ra, w;
+};
+
+// Delta lane: decode head h of its stream in steps of 8 values.
+__device__ __forceinline__ void decode_delta_head(uint32_t& x, Pos& ps, Ring& r,
+                                                  const uint32_t* __restrict__ tbl, float step,
                                                   const float* __restrict__ arow,
-                                                  uint16_t* __restrict__ orow, int D,
-                                                  const uint16_t* __restrict__ w16,
-                                                  uint64_t limit) {
+                                                  uint16_t* __restrict__ orow, int D) {
   for (int d0 = 0; d0 < D; d0 += 8) {
+    ring_issue(r, ps.p);
+    ring_wait_two_steps();
+    const uint32_t ra0 = ps.ra;
     const float4 a0 = *reinterpret_cast<const float4*>(arow + d0);
     const float4 a1 = *reinterpret_cast<const float4*>(arow + d0 + 4);
     const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     uint32_t hv[4];
 #pragma unroll
     for (int k = 0; k < 8; k += 2) {
-      const uint32_t e0 = rans_step<kClamp>(x, p, w, tbl, w16, limit);
-      const float v0 = __fadd_rn(a[k], lut[(e0 >> 12) & 0xFF]);
-      const uint32_t e1 = rans_step<kClamp>(x, p, w, tbl, w16, limit);
-      const float v1 = __fadd_rn(a[k + 1], lut[(e1 >> 12) & 0xFF]);
+      const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+      const float v0 = __fadd_rn(a[k], __fmul_rn(sym_value(e0), step));
+      const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+      const float v1 = __fadd_rn(a[k + 1], __fmul_rn(sym_value(e1), step));
       hv[k >> 1] = pack_half2(v0, v1);
     }
+    ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
     *reinterpret_cast<uint4*>(orow + d0) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
   }
 }
 
 // Anchor lane: decode head h, write fp16(a) and keep a (fp32) for the deltas.
-template <bool kClamp>
-__device__ __forceinline__ void decode_anchor_head(uint32_t& x, uint64_t& p, uint32_t& w,
+// zp and sc point at the head's zero points and scales staged in shared memory.
+__device__ __forceinline__ void decode_anchor_head(uint32_t& x, Pos& ps, Ring& r,
                                                    const uint32_t* __restrict__ tbl,
                                                    const float* __restrict__ zp,
                                                    const float* __restrict__ sc,
                                                    float* __restrict__ arow,
-                                                   uint16_t* __restrict__ orow, int D,
-                                                   const uint16_t* __restrict__ w16,
-                                                   uint64_t limit) {
+                                                   uint16_t* __restrict__ orow, int D) {
   for (int d0 = 0; d0 < D; d0 += 8) {
-    const float4 z0 = __ldg(reinterpret_cast<const float4*>(zp + d0));
-    const float4 z1 = __ldg(reinterpret_cast<const float4*>(zp + d0 + 4));
-    const float4 s0 = __ldg(reinterpret_cast<const float4*>(sc + d0));
-    const float4 s1 = __ldg(reinterpret_cast<const float4*>(sc + d0 + 4));
+    ring_issue(r, ps.p);
+    ring_wait_two_steps();
+    const uint32_t ra0 = ps.ra;
+    const float4 z0 = *reinterpret_cast<const float4*>(zp + d0);
+    const float4 z1 = *reinterpret_cast<const float4*>(zp + d0 + 4);
+    const float4 s0 = *reinterpret_cast<const float4*>(sc + d0);
+    const float4 s1 = *reinterpret_cast<const float4*>(sc + d0 + 4);
     const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
     const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
     float v[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint32_t e = rans_step<kClamp>(x, p, w, tbl, w16, limit);
-      const int c = int((e >> 12) & 0xFF) - 127;
-      v[k] = __fadd_rn(z[k], __fmul_rn(float(c), s[k]));
+      const uint32_t e = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+      v[k] = __fadd_rn(z[k], __fmul_rn(sym_value(e), s[k]));
     }
+    ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
     *reinterpret_cast<float4*>(arow + d0) = make_float4(v[0], v[1], v[2], v[3]);
     *reinterpret_cast<float4*>(arow + d0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
     *reinterpret_cast<uint4*>(orow + d0) =
@@ -224,49 +369,28 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   const DecSmem sm = dec_smem(H, D);
   uint32_t* tbl = reinterpret_cast<uint32_t*>(smem + sm.tbl);
   float* ahat = reinterpret_cast<float*>(smem + sm.ahat);
-  uint16_t* cum = reinterpret_cast<uint16_t*>(smem + sm.cum);
-  float* lut = reinterpret_cast<float*>(smem + sm.lut);
   int* single = reinterpret_cast<int*>(smem + sm.single);
   const int astride = D + 4;
   const int warp = tid >> 5, lane = tid & 31;
   const int slab = l * 2 + kv;
 
-  // Cumulative frequencies of every head of this (l, kv): warp-wide scans.
+  // Validate every frequency table of this (l, kv) and note one-symbol tables.
   const uint16_t* freq = reinterpret_cast<const uint16_t*>(base + sec.freq) + size_t(slab) * H * 256;
   for (int h = warp; h < H; h += kWarps) {
     const uint4 raw = __ldg(reinterpret_cast<const uint4*>(freq + h * 256) + lane);
     const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-    uint32_t f[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = wv[i] & 0xFFFF;
-      f[2 * i + 1] = wv[i] >> 16;
-    }
     uint32_t local = 0;
     int one = -1;
     bool bad = false;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      local += f[i];
-      if (f[i] == kM) one = lane * 8 + i;
-      if (f[i] > kM) bad = true;
+      const uint32_t f = (wv[i >> 1] >> (16 * (i & 1))) & 0xFFFF;
+      local += f;
+      if (f == kM) one = lane * 8 + i;
+      if (f > kM) bad = true;
     }
-    if (lane == 31 && f[7] != 0) bad = true;  // symbol 255 never exists
-    uint32_t incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-    uint32_t run = incl - local;
-    uint16_t* ch = cum + h * kCumStride;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      ch[lane * 8 + i] = uint16_t(run < kM ? run : kM);
-      run += f[i];
-    }
-    if (lane == 31) ch[256] = uint16_t(kM);
+    if (lane == 31 && (wv[3] >> 16) != 0) bad = true;  // symbol 255 never exists
+    const uint32_t total = __reduce_add_sync(0xFFFFFFFFu, local);
     one = __reduce_max_sync(0xFFFFFFFFu, one);
     if (lane == 0) single[h] = one;
     if (__any_sync(0xFFFFFFFFu, bad) || total != kM) {
@@ -274,13 +398,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
     }
   }
   const float step = step_of(p.level, l, L);
-  for (int u = tid; u < 256; u += kThreads) lut[u] = __fmul_rn(float(u - 127), step);
   __syncthreads();
   if (s_bad) {
     if (tid == 0) set_status(p.status, CG_ERR_CORRUPT);
     return;
   }
-  fill_table(tbl, cum, tid);
+  uint8_t* cumb = smem + sm.cum;
+  if (warp < 2 && warp < H)
+    cum_compact(__ldg(reinterpret_cast<const uint4*>(freq + warp * 256) + lane),
+                cum_buf(cumb + warp * kCumBuf), lane);
+  __syncthreads();
+  fill_table(tbl, cum_buf(cumb), tid);
 
   // This thread's stream.
   int g_local, token;
@@ -293,11 +421,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
     token = unit_t0 + kGroup * g_local + 1 + k % kDeltaPerGroup;
   }
   bool active = token < n;
-  const uint16_t* w16 = reinterpret_cast<const uint16_t*>(base);
-  const uint64_t limit = s_total / 2;  // u16 words readable in this container
   const uint32_t* offs = reinterpret_cast<const uint32_t*>(base + sec.offsets);
-  uint64_t pw = 0, pend = 0;
-  uint32_t x = kRansL, w = 0;
+  Ring ring;
+  ring.gbase = base;
+  const uint32_t rings = (uint32_t(__cvta_generic_to_shared(smem + sm.ring)) + 63u) & ~63u;
+  ring.rb = rings + uint32_t(tid) * kRingBytes;
+  ring.lim = uint32_t(s_total / 16);
+  ring.fb = 0;
+  Pos ps{0u, ring.rb, 0u};
+  uint32_t pend = 0, x = kRansL;
   if (active) {
     const uint64_t s = uint64_t(slab) * n + token;
     const uint32_t o0 = __ldg(offs + s), o1 = __ldg(offs + s + 1);
@@ -306,11 +438,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
       set_status(p.status, CG_ERR_CORRUPT);
       active = false;
     } else {
-      pw = (sec.payload + o0) / 2;
-      pend = (sec.payload + o1) / 2;
-      x = (uint32_t(ldg_u16(w16 + pw)) << 16) | ldg_u16(w16 + pw + 1);
+      uint32_t pw = uint32_t((sec.payload + o0) / 2);
+      pend = uint32_t((sec.payload + o1) / 2);
+      ring.fb = pw >> 3;
+      for (uint32_t i = 0; i < kRingBlocks; ++i) ring_issue(ring, pw);
+      ring_wait_all();
+      x = (lds_u16(ring_addr(ring, pw)) << 16) | lds_u16(ring_addr(ring, pw + 1));
       pw += 2;
-      w = pw < limit ? ldg_u16(w16 + pw) : 0;
+      ps.p = pw;
+      ps.ra = ring_addr(ring, pw);
+      ps.w = lds_u16(ps.ra);
       if (x < kRansL) {
         set_status(p.status, CG_ERR_CORRUPT);
         active = false;
@@ -325,35 +462,49 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
            ((uint64_t(slab) * n + token) * H) * D;
   const float* zp_sec = reinterpret_cast<const float*>(base + sec.zp) + size_t(slab) * H * D;
   const float* sc_sec = reinterpret_cast<const float*>(base + sec.scale) + size_t(slab) * H * D;
+  float* zs = reinterpret_cast<float*>(smem + sm.zs);  // [2][{zp, scale}][D]
+  for (int i = tid; i < 2 * D; i += kThreads)
+    zs[i] = i < D ? __ldg(zp_sec + i) : __ldg(sc_sec + (i - D));
   __syncthreads();
 
   for (int it = 0; it <= H; ++it) {
-    if (it + 1 < H) fill_table(tbl + ((it + 1) % 3) * kM, cum + (it + 1) * kCumStride, tid);
+    // Global loads for the next heads are issued first and consumed after this
+    // iteration's decode, so their latency never delays the barrier.
+    const bool scan_warp = it + 2 < H && warp == it % kWarps;
+    uint4 fq = make_uint4(0, 0, 0, 0);
+    if (scan_warp) fq = __ldg(reinterpret_cast<const uint4*>(freq + (it + 2) * 256) + lane);
+    float zv[2] = {0.0f, 0.0f};
+    const bool stage = it + 1 < H;
+    if (stage) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int i = tid + j * kThreads;
+        if (i < 2 * D)
+          zv[j] = i < D ? __ldg(zp_sec + (it + 1) * D + i) : __ldg(sc_sec + (it + 1) * D + (i - D));
+      }
+      fill_table(tbl + ((it + 1) % 3) * kM, cum_buf(cumb + ((it + 1) & 1) * kCumBuf), tid);
+    }
     if (warp == 0) {
       if (it < H && active) {
         const int h = it;
         const uint32_t* tb = tbl + (h % 3) * kM;
         float* arow = ahat + ((h & 1) * kUnitGroups + g_local) * astride;
+        const float* zh = zs + (h & 1) * 2 * D;
         const int one = single[h];
         if (one >= 0) {
           const float c = float(one - 127);
           for (int d0 = 0; d0 < D; d0 += 8) {
             float v[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              v[k] = __fadd_rn(zp_sec[h * D + d0 + k], __fmul_rn(c, sc_sec[h * D + d0 + k]));
+            for (int k = 0; k < 8; ++k) v[k] = __fadd_rn(zh[d0 + k], __fmul_rn(c, zh[D + d0 + k]));
 #pragma unroll
             for (int k = 0; k < 8; ++k) arow[d0 + k] = v[k];
             *reinterpret_cast<uint4*>(orow + h * D + d0) =
                 make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]),
                            pack_half2(v[4], v[5]), pack_half2(v[6], v[7]));
           }
-        } else if (pw + uint64_t(D) + 1 <= limit) {
-          decode_anchor_head<false>(x, pw, w, tb, zp_sec + h * D, sc_sec + h * D, arow,
-                                    orow + h * D, D, w16, limit);
         } else {
-          decode_anchor_head<true>(x, pw, w, tb, zp_sec + h * D, sc_sec + h * D, arow,
-                                   orow + h * D, D, w16, limit);
+          decode_anchor_head(x, ps, ring, tb, zh, zh + D, arow, orow + h * D, D);
         }
       }
     } else if (it >= 1 && active) {
@@ -362,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
       const float* arow = ahat + ((h & 1) * kUnitGroups + g_local) * astride;
       const int one = single[h];
       if (one >= 0) {
-        const float v = lut[one];
+        const float v = __fmul_rn(float(one - 127), step);
         for (int d0 = 0; d0 < D; d0 += 8) {
           uint32_t hv[4];
 #pragma unroll
@@ -370,29 +521,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
             hv[k >> 1] = pack_half2(__fadd_rn(arow[d0 + k], v), __fadd_rn(arow[d0 + k + 1], v));
           *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
-      } else if (pw + uint64_t(D) + 1 <= limit) {
-        decode_delta_head<false>(x, pw, w, tb, lut, arow, orow + h * D, D, w16, limit);
       } else {
-        decode_delta_head<true>(x, pw, w, tb, lut, arow, orow + h * D, D, w16, limit);
+        decode_delta_head(x, ps, ring, tb, step, arow, orow + h * D, D);
+      }
+    }
+    if (scan_warp) cum_compact(fq, cum_buf(cumb + (it & 1) * kCumBuf), lane);
+    if (stage) {
+      float* zn = zs + ((it + 1) & 1) * 2 * D;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int i = tid + j * kThreads;
+        if (i < 2 * D) zn[i] = zv[j];
       }
     }
     __syncthreads();
   }
-  if (active && (x != kRansL || pw != pend)) set_status(p.status, CG_ERR_CORRUPT);
+  ring_wait_all();
+  if (active && (x != kRansL || ps.p != pend)) set_status(p.status, CG_ERR_CORRUPT);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecParams& p, cudaStream_t stream) {
   const DecSmem sm = dec_smem(p.H, p.D);
-  static thread_local int configured_bytes = -1;
-  cudaError_t err = cudaSuccess;
-  if (configured_bytes < int(sm.total)) {
-    err = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(sm.total));
-    if (err != cudaSuccess) return err;
-    configured_bytes = int(sm.total);
-  }
+  cudaError_t err = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(sm.total));
+  if (err != cudaSuccess) return err;
   const uint64_t blocks = uint64_t(p.num_chunks) * p.L * 2 * p.units_per_slab;
   decode_kernel<<<unsigned(blocks), kThreads, sm.total, stream>>>(p);
   return cudaGetLastError();

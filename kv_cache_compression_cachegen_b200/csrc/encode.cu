@@ -17,8 +17,10 @@
 //                   renormalisation words go through a per-thread ring in
 //                   shared memory and leave in 32-byte blocks, written
 //                   backwards into a per-stream scratch slot.
-//   scan_kernel     one CTA per chunk: exclusive prefix sum of stream lengths
-//                   -> offsets section, header, container size.
+//   offsets_kernel  one CTA per (chunk, layer, K/V): its base (the words of the
+//                   earlier layers, summed by the rANS pass) plus an exclusive
+//                   scan of its stream lengths -> offsets; the last one of a
+//                   chunk writes the header and the container size.
 //   compact_kernel  one warp per stream: scratch slot -> payload.
 #include <cuda_fp16.h>
 
@@ -28,11 +30,14 @@ namespace cg {
 namespace {
 
 constexpr int kQThreads = 256;
+constexpr int kSlots = 3;                          // token slots in flight per thread (6 x 16 B)
 constexpr int kTileGroups = 16;
 constexpr int kTileTokens = kTileGroups * kGroup;  // 160
 constexpr int kRThreads = 128;                     // rANS streams per CTA
 constexpr int kRing = 64;                          // u16 ring entries per thread
-constexpr int kScanThreads = 1024;
+constexpr int kRingStride = 72;                    // u16; 144 B keeps 16-B alignment and
+                                                   // staggers the threads' banks
+constexpr int kScanThreads = 256;
 
 enum QuantMode { kModeEncode = 0, kModeTablesOnly = 1, kModeSuppliedTables = 2 };
 
@@ -41,9 +46,9 @@ struct QSmem {
   uint32_t zp;      // f32 [256]
   uint32_t sc;      // f32 [256]
   uint32_t rcp;     // f32 [256]
-  uint32_t ahat;    // f32 [16][D + 4]
-  uint32_t red;     // f32 [2][512]   range reduction
-  uint32_t counts;  // u32 [256]
+  uint32_t ahat;    // f32 [16][D + 4]  (phase B)
+  uint32_t red;     // f32 [2][512]     range reduction (phase A, aliases ahat)
+  uint32_t counts;  // u32 [256]        histogram totals (phase C, aliases ahat)
   uint32_t total;
 };
 
@@ -56,9 +61,12 @@ __host__ __device__ inline QSmem q_smem(int D) {
   s.sc = s.zp + 1024u;
   s.rcp = s.sc + 1024u;
   s.ahat = s.rcp + 1024u;
-  s.red = a16(s.ahat + uint32_t(kTileGroups) * uint32_t(D + 4) * 4u);
-  s.counts = s.red + 2u * 512u * 4u;
-  s.total = a16(s.counts + 256u * 4u);
+  // red (phase A) and counts (phase C) reuse the anchor buffer of phase B
+  s.red = s.ahat;
+  s.counts = s.ahat;
+  const uint32_t ahat_bytes = uint32_t(kTileGroups) * uint32_t(D + 4) * 4u;
+  const uint32_t red_bytes = 2u * 512u * 4u;
+  s.total = a16(s.ahat + (ahat_bytes > red_bytes ? ahat_bytes : red_bytes));
   return s;
 }
 
@@ -183,20 +191,25 @@ __device__ void normalize_warp(const uint32_t* counts, uint64_t N, uint32_t f[8]
   }
 }
 
-// Encoder constants of one symbol: x_max - 1, the Granlund-Montgomery
-// multiplier for exact 32-bit division by f ("Division by invariant integers
-// using multiplication", 1994, the N+1-bit case), cum, 4096 - f and the shifts.
+// Encoder constants of one symbol.  The state stays in [2^15, 2^31), so
+// floor(x / f) = umulhi(2x, m) >> l with l = ceil(log2 f) and the 32-bit
+// multiplier m = ceil(2^(31+l) / f) (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994, theorem 4.2 with N = 31).
+//   .x = (f << 19) - 1   the largest state that needs no renormalisation
+//   .y = m
+//   .z = cum
+//   .w = ((4096 - f) << 5) | l   (a funnel shift reads l from the low 5 bits)
+// Sixteen bytes per entry keep the per-symbol arithmetic minimal; an absent
+// symbol (f == 0) gets .w = 0xFFFFFFFF, which no present symbol has.
 __device__ __forceinline__ uint4 enc_entry(uint32_t f, uint32_t cum) {
-  if (f == 0) return make_uint4(0xFFFFFFFFu, 0u, 0u, 0u);
+  if (f == 0) return make_uint4(0xFFFFFFFFu, 0u, 0u, 0xFFFFFFFFu);
   const uint32_t lg = f == 1 ? 0u : 32u - __clz(f - 1);  // ceil(log2 f)
-  const uint32_t magic =
-      uint32_t(((1ull << 32) * ((1ull << lg) - f)) / f + 1ull);
-  const uint32_t sh1 = lg < 1 ? lg : 1u;
-  const uint32_t sh2 = lg > 0 ? lg - 1 : 0u;
-  return make_uint4((f << 20) - 1u, magic, cum | ((kM - f) << 16), sh1 | (sh2 << 8) | (f << 16));
+  const uint64_t num = 1ull << (31 + lg);
+  const uint32_t magic = uint32_t((num + f - 1) / f);
+  return make_uint4((f << 19) - 1u, magic, cum, ((kM - f) << 5) | lg);
 }
 
-__global__ void __launch_bounds__(kQThreads) quant_kernel(const EncParams p, const int mode) {
+__global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const EncParams p, const int mode) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int rest = blockIdx.x;
@@ -235,6 +248,7 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const EncParams p, con
 
   if (want_hist)
     for (int i = tid; i < kAlphabet * 32; i += kQThreads) hist[i] = 0;
+  if (want_sym && h == 0 && tid == 0) p.slabtot[uint64_t(chunk) * L * 2 + slab] = 0;
 
   // ---- Phase A: per-channel anchor range -> zp, scale (or the supplied ones).
   bool nonfinite = false;
@@ -250,16 +264,25 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const EncParams p, con
     const int pi = tid % np, r = tid / np;
     float lo0 = __int_as_float(0x7F800000), hi0 = -lo0, lo1 = lo0, hi1 = hi0;
     if (r < rp) {
-      for (int g = r; g < Gn; g += rp) {
-        const uint32_t v =
-            __ldg(reinterpret_cast<const uint32_t*>(col + uint64_t(g) * kGroup * rs) + pi);
-        const float a = half_bits_to_float(uint16_t(v & 0xFFFF));
-        const float b = half_bits_to_float(uint16_t(v >> 16));
-        if (!isfinite(a) || !isfinite(b)) nonfinite = true;
-        lo0 = fminf(lo0, a);
-        hi0 = fmaxf(hi0, a);
-        lo1 = fminf(lo1, b);
-        hi1 = fmaxf(hi1, b);
+      for (int g0 = r; g0 < Gn; g0 += 8 * rp) {  // eight anchor rows in flight
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int g = g0 + j * rp;
+          v[j] = g < Gn ? __ldg(reinterpret_cast<const uint32_t*>(col + uint64_t(g) * kGroup * rs) + pi)
+                        : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (g0 + j * rp >= Gn) continue;
+          const float a = half_bits_to_float(uint16_t(v[j] & 0xFFFF));
+          const float b = half_bits_to_float(uint16_t(v[j] >> 16));
+          if (!isfinite(a) || !isfinite(b)) nonfinite = true;
+          lo0 = fminf(lo0, a);
+          hi0 = fmaxf(hi0, a);
+          lo1 = fminf(lo1, b);
+          hi1 = fmaxf(hi1, b);
+        }
       }
       red[r * D + 2 * pi] = lo0;
       red[r * D + 2 * pi + 1] = lo1;
@@ -304,69 +327,105 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const EncParams p, con
   for (int tb = 0; tb < n; tb += kTileTokens) {
     const int g0 = tb / kGroup;
     const int ng = min(kTileGroups, Gn - g0);
-    // B1: anchor codes and reconstructed anchors of the tile's groups.
-    for (int idx = tid; idx < ng * D; idx += kQThreads) {
-      const int gi = idx / D, d = idx - gi * D;
+    // B1: anchor codes and reconstructed anchors of the tile's groups, eight
+    // channels (one 16-byte load) per thread.
+    for (int idx = tid; idx < ng * (D / 8); idx += kQThreads) {
+      const int gi = idx / (D / 8), d = (idx - gi * (D / 8)) * 8;
       const int t = tb + kGroup * gi;
-      const float x = half_bits_to_float(__ldg(col + uint64_t(t) * rs + d));
-      if (!isfinite(x)) nonfinite = true;
-      bool ok = true;
-      uint32_t u = quant_fast(__fsub_rn(x, zp[d]), rcp[d], ok);
-      if (!ok) u = quant_exact(x, zp[d], sc[d]);
-      const int c = int(u) - 127;
-      ahat[gi * astride + d] = __fadd_rn(zp[d], __fmul_rn(float(c), sc[d]));
-      if (want_hist) atomicAdd(&hist[u * 32 + lane], 1u);
-      if (want_sym) symc[(uint64_t(d >> 4) * C + t) * 16 + (d & 15)] = uint8_t(u);
+      const uint4 rv = __ldg(reinterpret_cast<const uint4*>(col + uint64_t(t) * rs + d));
+      const uint32_t raw[4] = {rv.x, rv.y, rv.z, rv.w};
+      uint32_t u[8];
+      float av[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q]));
+        const float xs[2] = {f2.x, f2.y};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int dd = d + 2 * q + e;
+          const float x = xs[e];
+          if (!isfinite(x)) nonfinite = true;
+          bool ok = true;
+          uint32_t uu = quant_fast(__fsub_rn(x, zp[dd]), rcp[dd], ok);
+          if (!ok) uu = quant_exact(x, zp[dd], sc[dd]);
+          u[2 * q + e] = uu;
+          av[2 * q + e] = __fadd_rn(zp[dd], __fmul_rn(float(int(uu) - 127), sc[dd]));
+        }
+      }
+      *reinterpret_cast<float4*>(ahat + gi * astride + d) = make_float4(av[0], av[1], av[2], av[3]);
+      *reinterpret_cast<float4*>(ahat + gi * astride + d + 4) =
+          make_float4(av[4], av[5], av[6], av[7]);
+      if (want_hist) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) atomicAdd(&hist[u[q] * 32 + lane], 1u);
+      }
+      if (want_sym)
+        *reinterpret_cast<uint2*>(symc + (uint64_t(d >> 4) * C + t) * 16 + (d & 15)) =
+            make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
+                       u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
     }
     __syncthreads();
-    // B2: the delta tokens of the tile; lane -> (token slot, 16-value block).
+    // B2: the delta tokens of the tile; lane -> (token slot, 16-value block),
+    // kSlots token slots per pass so that 2 * kSlots 16-byte loads are in flight.
     if (lane_ok) {
-      for (int k = warp * tpw + tw; k < ng * (kGroup - 1); k += (kQThreads / 32) * tpw) {
-        const int gi = k / (kGroup - 1);
-        const int t = tb + kGroup * gi + 1 + (k - gi * (kGroup - 1));
-        if (t >= n) continue;
-        const uint4* src = reinterpret_cast<const uint4*>(col + uint64_t(t) * rs + 16 * b);
-        const uint4 r0 = __ldg(src), r1 = __ldg(src + 1);
-        const uint32_t raw[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-        const float4* ap = reinterpret_cast<const float4*>(ahat + gi * astride + 16 * b);
-        float a[16];
+      const int kslots = ng * (kGroup - 1);
+      const int kstride = (kQThreads / 32) * tpw;
+      for (int k = warp * tpw + tw; k < kslots; k += kSlots * kstride) {
+        int gi[kSlots], tk[kSlots];
+        bool has[kSlots];
+        uint4 r[kSlots][2];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 v = ap[j];
-          a[4 * j] = v.x;
-          a[4 * j + 1] = v.y;
-          a[4 * j + 2] = v.z;
-          a[4 * j + 3] = v.w;
-        }
-        float x[16];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[j]));
-          x[2 * j] = f2.x;
-          x[2 * j + 1] = f2.y;
-        }
-        bool ok = true;
-        uint32_t u[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) u[j] = quant_fast(__fsub_rn(x[j], a[j]), rstep, ok);
-        if (!ok) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (!isfinite(x[j])) nonfinite = true;
-            u[j] = quant_exact(x[j], a[j], step);
+        for (int j = 0; j < kSlots; ++j) {
+          const int kk = k + j * kstride;
+          gi[j] = kk / (kGroup - 1);
+          tk[j] = tb + kGroup * gi[j] + 1 + (kk - gi[j] * (kGroup - 1));
+          has[j] = kk < kslots && tk[j] < n;
+          if (has[j]) {
+            const uint4* src = reinterpret_cast<const uint4*>(col + uint64_t(tk[j]) * rs + 16 * b);
+            r[j][0] = __ldg(src);
+            r[j][1] = __ldg(src + 1);
           }
         }
-        if (want_hist) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) atomicAdd(&hist[u[j] * 32 + lane], 1u);
-        }
-        if (want_sym) {
+        for (int j = 0; j < kSlots; ++j) {
+          if (!has[j]) continue;
+          const float* arow = ahat + gi[j] * astride + 16 * b;
           uint32_t pk[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            pk[j] = u[4 * j] | (u[4 * j + 1] << 8) | (u[4 * j + 2] << 16) | (u[4 * j + 3] << 24);
-          *reinterpret_cast<uint4*>(symc + (uint64_t(b) * C + t) * 16) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          for (int half = 0; half < 2; ++half) {  // 8 values at a time keeps registers low
+            const uint4 rv = r[j][half];
+            const uint32_t raw[4] = {rv.x, rv.y, rv.z, rv.w};
+            const float4 av0 = *reinterpret_cast<const float4*>(arow + 8 * half);
+            const float4 av1 = *reinterpret_cast<const float4*>(arow + 8 * half + 4);
+            const float a[8] = {av0.x, av0.y, av0.z, av0.w, av1.x, av1.y, av1.z, av1.w};
+            float x[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q]));
+              x[2 * q] = f2.x;
+              x[2 * q + 1] = f2.y;
+            }
+            bool ok = true;
+            uint32_t u[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) u[q] = quant_fast(__fsub_rn(x[q], a[q]), rstep, ok);
+            if (!ok) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                if (!isfinite(x[q])) nonfinite = true;
+                u[q] = quant_exact(x[q], a[q], step);
+              }
+            }
+            if (want_hist) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) atomicAdd(&hist[u[q] * 32 + lane], 1u);
+            }
+            pk[2 * half] = u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24);
+            pk[2 * half + 1] = u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24);
+          }
+          if (want_sym)
+            *reinterpret_cast<uint4*>(symc + (uint64_t(b) * C + tk[j]) * 16) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
       }
     }
@@ -426,9 +485,38 @@ __global__ void __launch_bounds__(kQThreads) quant_kernel(const EncParams p, con
 
 __device__ __forceinline__ uint32_t swap16(uint32_t v) { return __byte_perm(v, 0, 0x1032); }
 
-__global__ void __launch_bounds__(kRThreads, 4) rans_kernel(const EncParams p, const int check_f) {
-  __shared__ __align__(16) uint4 et[256];
-  __shared__ __align__(16) uint16_t ring[kRThreads * kRing];
+// One rANS encoder step with the constants e of the symbol (see enc_entry):
+// renormalise by pushing the low 16 bits into the thread's ring when
+// x > (f << 19) - 1, then x = floor(x / f) * 4096 + x mod f + cum computed as
+// x + cum + q * (4096 - f).  Predicated rather than branched; the asm does not
+// clobber memory, so the caller orders the ring reads with a compiler barrier.
+__device__ __forceinline__ void enc_step(uint32_t& x, uint32_t& wp, uint32_t ring_s,
+                                         const uint4& e) {
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      ".reg .u32 a, t, q;\n\t"
+      "setp.gt.u32 p, %0, %3;\n\t"
+      "@p and.b32 a, %1, 63;\n\t"
+      "@p mad.lo.u32 a, a, 2, %2;\n\t"
+      "@p st.shared.u16 [a], %0;\n\t"
+      "@p add.u32 %1, %1, 1;\n\t"
+      "@p shr.u32 %0, %0, 16;\n\t"
+      "add.u32 t, %0, %0;\n\t"
+      "mul.hi.u32 t, t, %4;\n\t"
+      "shf.r.wrap.b32 q, t, 0, %6;\n\t"
+      "shr.u32 t, %6, 5;\n\t"
+      "add.u32 %0, %0, %5;\n\t"
+      "mad.lo.u32 %0, q, t, %0;\n\t"
+      "}\n"
+      : "+r"(x), "+r"(wp)
+      : "r"(ring_s), "r"(e.x), "r"(e.y), "r"(e.z), "r"(e.w));
+}
+
+template <bool kCheckF>
+__global__ void __launch_bounds__(kRThreads, 6) rans_kernel(const EncParams p) {
+  __shared__ __align__(16) uint4 et[2][256];
+  __shared__ __align__(16) uint16_t ring[kRThreads * kRingStride];
   const int tid = threadIdx.x;
   const int C = p.C, L = p.L, H = p.H, D = p.D;
   const int tiles = (C + kRThreads - 1) / kRThreads;
@@ -444,102 +532,140 @@ __global__ void __launch_bounds__(kRThreads, 4) rans_kernel(const EncParams p, c
   const int nb = D / 16;
   const uint64_t cs = uint64_t(chunk) * L * 2 + slab;
   const uint4* etg = reinterpret_cast<const uint4*>(p.etab) + cs * H * 256;
-  const uint8_t* symc = p.sym + cs * H * uint64_t(nb) * C * 16;
+  // symbols of this token, 16-byte blocks ordered (h, b); block index h*nb + b
+  const uint4* symt = reinterpret_cast<const uint4*>(p.sym + cs * H * uint64_t(nb) * C * 16) + t;
   const uint64_t ss = scratch_stride(H, D);
-  uint16_t* rend = reinterpret_cast<uint16_t*>(p.scratch + (cs * C + t + 1) * ss);
-  uint16_t* myring = ring + tid * kRing;
+  uint16_t* rend = active ? reinterpret_cast<uint16_t*>(p.scratch + (cs * C + t + 1) * ss) : nullptr;
+  uint16_t* myring = ring + tid * kRingStride;
+  const uint32_t ring_s = uint32_t(__cvta_generic_to_shared(myring));
 
+  // Stage the last head's encoder table; prefetch the next one into registers.
+  et[(H - 1) & 1][tid] = __ldg(etg + uint64_t(H - 1) * 256 + tid);
+  et[(H - 1) & 1][tid + kRThreads] = __ldg(etg + uint64_t(H - 1) * 256 + tid + kRThreads);
   uint32_t x = kRansL, wp = 0, wf = 0;
   bool bad = false;
+  int blk = H * nb - 1;  // next 16-symbol block, walking backwards
+  uint4 vnext = active ? __ldg(symt + uint64_t(blk) * C) : make_uint4(0, 0, 0, 0);
   for (int h = H - 1; h >= 0; --h) {
-    __syncthreads();
-    et[tid] = __ldg(etg + uint64_t(h) * 256 + tid);
-    et[tid + kRThreads] = __ldg(etg + uint64_t(h) * 256 + tid + kRThreads);
-    __syncthreads();
-    if (!active) continue;
-    for (int b = nb - 1; b >= 0; --b) {
-      const uint4 v =
-          __ldg(reinterpret_cast<const uint4*>(symc + ((uint64_t(h) * nb + b) * C + t) * 16));
+    uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+    if (h > 0) {
+      n0 = __ldg(etg + uint64_t(h - 1) * 256 + tid);
+      n1 = __ldg(etg + uint64_t(h - 1) * 256 + tid + kRThreads);
+    }
+    __syncthreads();  // table h is staged; nobody reads buffer (h+1)&1 any more
+    const uint4* eh = et[h & 1];
+    if (active) {
+      for (int b = nb - 1; b >= 0; --b, --blk) {
+        const uint4 v = vnext;
+        if (blk > 0) vnext = __ldg(symt + uint64_t(blk - 1) * C);
 #pragma unroll
-      for (int k = 15; k >= 0; --k) {
-        const uint32_t word = (k >> 2) == 0 ? v.x : (k >> 2) == 1 ? v.y : (k >> 2) == 2 ? v.z : v.w;
-        const uint32_t u = (word >> (8 * (k & 3))) & 0xFFu;
-        const uint4 e = et[u];
-        if (x > e.x) {
-          myring[wp & (kRing - 1)] = uint16_t(x);
-          ++wp;
-          x >>= 16;
+        for (int k = 15; k >= 0; --k) {
+          const uint32_t word = (k >> 2) == 0 ? v.x : (k >> 2) == 1 ? v.y : (k >> 2) == 2 ? v.z : v.w;
+          const uint32_t u = (word >> (8 * (k & 3))) & 0xFFu;
+          const uint4 e = eh[u];
+          enc_step(x, wp, ring_s, e);
+          if (kCheckF) bad |= e.w == 0xFFFFFFFFu;
         }
-        const uint32_t t1 = __umulhi(x, e.y);
-        const uint32_t q = (t1 + ((x - t1) >> (e.w & 0xFFu))) >> ((e.w >> 8) & 0xFFu);
-        x = x + (e.z & 0xFFFFu) + q * (e.z >> 16);
-        if (check_f) bad |= (e.w >> 16) == 0u;
-      }
-      if (wp - wf >= 16) {
-        const uint4* src = reinterpret_cast<const uint4*>(myring + (wf & (kRing - 1)));
-        const uint4 r0 = src[0], r1 = src[1];
-        uint4* dst = reinterpret_cast<uint4*>(rend - wf - 16);
-        dst[0] = make_uint4(swap16(r1.w), swap16(r1.z), swap16(r1.y), swap16(r1.x));
-        dst[1] = make_uint4(swap16(r0.w), swap16(r0.z), swap16(r0.y), swap16(r0.x));
-        wf += 16;
+        // the ring stores inside enc_step precede the ring reads of the flush
+        asm volatile("" ::: "memory");
+        if (wp - wf >= 16) {
+          const uint4* src = reinterpret_cast<const uint4*>(myring + (wf & (kRing - 1)));
+          const uint4 r0 = src[0], r1 = src[1];
+          uint4* dst = reinterpret_cast<uint4*>(rend - wf - 16);
+          dst[0] = make_uint4(swap16(r1.w), swap16(r1.z), swap16(r1.y), swap16(r1.x));
+          dst[1] = make_uint4(swap16(r0.w), swap16(r0.z), swap16(r0.y), swap16(r0.x));
+          wf += 16;
+        }
       }
     }
+    if (h > 0) {
+      et[(h - 1) & 1][tid] = n0;
+      et[(h - 1) & 1][tid + kRThreads] = n1;
+    }
   }
-  if (!active) return;
-  myring[wp & (kRing - 1)] = uint16_t(x);
-  ++wp;
-  myring[wp & (kRing - 1)] = uint16_t(x >> 16);
-  ++wp;
-  for (uint32_t k = wf; k < wp; ++k) rend[-1 - int64_t(k)] = myring[k & (kRing - 1)];
-  p.lens[cs * C + t] = wp;
-  if (bad) set_status(p.status, CG_ERR_MISMATCH);
+  asm volatile("" ::: "memory");
+  if (active) {
+    myring[wp & (kRing - 1)] = uint16_t(x);
+    ++wp;
+    myring[wp & (kRing - 1)] = uint16_t(x >> 16);
+    ++wp;
+    for (uint32_t k = wf; k < wp; ++k) rend[-1 - int64_t(k)] = myring[k & (kRing - 1)];
+    p.lens[cs * C + t] = wp;
+    if (kCheckF && bad) set_status(p.status, CG_ERR_MISMATCH);
+  }
+  // this CTA's share of the (layer, K/V) total, for the offsets pass
+  const uint32_t mine = __reduce_add_sync(0xFFFFFFFFu, active ? wp : 0u);
+  if ((tid & 31) == 0) atomicAdd(p.slabtot + cs, mine);
 }
 
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(const EncParams p) {
-  __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t s_total;
-  const int chunk = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int C = p.C, L = p.L, H = p.H, D = p.D;
-  const int64_t t0 = p.token_start + int64_t(chunk) * C;
-  const int n = int(min(int64_t(C), p.T - t0));
-  const Sections sec = sections(L, H, D, n);
-  uint8_t* cont = p.out + uint64_t(chunk) * p.out_stride;
-  uint32_t* offs = reinterpret_cast<uint32_t*>(cont + sec.offsets);
-  const uint32_t* lens = p.lens + uint64_t(chunk) * L * 2 * C;
-  const int S = 2 * L * n;
-  const int per = (S + kScanThreads - 1) / kScanThreads;
-  const int s0 = min(S, tid * per), s1 = min(S, s0 + per);
-  uint32_t local = 0;
-  for (int s = s0; s < s1; ++s) local += lens[(s / n) * C + (s % n)];
-  uint32_t incl = local;
+// Block-wide exclusive scan of one value per thread (kScanThreads threads).
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot,
+                                                         uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
+    const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += u;
   }
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t v = warp_tot[lane];
-    uint32_t wi = v;
+    const uint32_t t = lane < kScanThreads / 32 ? warp_tot[lane] : 0u;
+    uint32_t ti = t;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, wi, o);
-      if (lane >= o) wi += u;
+      const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, ti, o);
+      if (lane >= o) ti += u;
     }
-    warp_tot[lane] = wi - v;
-    if (lane == 31) s_total = wi;
+    if (lane < kScanThreads / 32) warp_tot[lane] = ti - t;
+    if (lane == 31) warp_tot[32] = ti;
   }
   __syncthreads();
-  uint32_t run = warp_tot[warp] + incl - local;  // words before this thread's range
+  total = warp_tot[32];
+  return warp_tot[warp] + incl - v;
+}
+
+// One CTA per (chunk, layer, K/V): the offsets of its streams are the words of
+// every earlier (layer, K/V) of the chunk plus an exclusive scan of its own
+// stream lengths.  The last (layer, K/V) of a chunk also writes the header.
+__global__ void __launch_bounds__(kScanThreads) offsets_kernel(const EncParams p) {
+  __shared__ uint32_t warp_tot[33];
+  const int tid = threadIdx.x;
+  const int C = p.C, L = p.L, H = p.H, D = p.D;
+  const int slab = blockIdx.x % (2 * L);
+  const int chunk = blockIdx.x / (2 * L);
+  const int64_t t0 = p.token_start + int64_t(chunk) * C;
+  const int n = int(min(int64_t(C), p.T - t0));
+  const Sections sec = sections(L, H, D, n);
+  uint8_t* cont = p.out + uint64_t(chunk) * p.out_stride;
+  uint32_t* offs = reinterpret_cast<uint32_t*>(cont + sec.offsets) + uint64_t(slab) * n;
+  const uint32_t* tot = p.slabtot + uint64_t(chunk) * L * 2;
+  const uint32_t* lens = p.lens + (uint64_t(chunk) * L * 2 + slab) * C;
+
+  uint32_t part = 0;
+  for (int i = tid; i < slab; i += kScanThreads) part += tot[i];
+  uint32_t base_total;
+  block_exclusive_scan(part, warp_tot, base_total);  // only the total is used
+  const uint32_t base = base_total;
+  __syncthreads();  // warp_tot is reused below
+
+  const int per = (n + kScanThreads - 1) / kScanThreads;
+  const int s0 = min(n, tid * per), s1 = min(n, s0 + per);
+  uint32_t local = 0;
+  for (int s = s0; s < s1; ++s) local += lens[s];
+  uint32_t slab_words;
+  uint32_t run = base + block_exclusive_scan(local, warp_tot, slab_words);
   for (int s = s0; s < s1; ++s) {
     offs[s] = 2u * run;
-    run += lens[(s / n) * C + (s % n)];
+    run += lens[s];
   }
-  const uint64_t payload = 2ull * s_total;
+  if (slab != 2 * L - 1) return;
+
+  const uint64_t payload = 2ull * (uint64_t(base) + slab_words);
+  const uint64_t total = up16(sec.payload + payload);
   if (tid == 0) {
-    offs[S] = uint32_t(payload);
-    const uint64_t total = up16(sec.payload + payload);
+    offs[n] = uint32_t(payload);  // == offsets[2 L n]
     cg_header hd;
     hd.magic = CG_MAGIC;
     hd.version = CG_FORMAT_VERSION;
@@ -561,9 +687,8 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const EncParams p) {
     if (total > p.out_stride) set_status(p.status, CG_ERR_CAPACITY);
   }
   // Zero the padding after the offsets section and after the payload.
-  const uint64_t opad0 = sec.offsets + 4ull * (uint64_t(S) + 1);
+  const uint64_t opad0 = sec.offsets + 4ull * (2ull * L * n + 1);
   if (tid < int(sec.payload - opad0)) cont[opad0 + tid] = 0;
-  const uint64_t total = up16(sec.payload + payload);
   const uint64_t ppad0 = sec.payload + payload;
   if (total <= p.out_stride && tid < int(total - ppad0)) cont[ppad0 + tid] = 0;
 }
@@ -589,7 +714,15 @@ __global__ void __launch_bounds__(256) compact_kernel(const EncParams p) {
   const uint16_t* src =
       reinterpret_cast<const uint16_t*>(p.scratch + (cs * C + t + 1) * scratch_stride(H, D)) - len;
   uint16_t* dst = reinterpret_cast<uint16_t*>(cont + sec.payload + o0);
-  for (uint32_t i = lane; i < len; i += 32) dst[i] = src[i];
+  uint32_t i = lane;
+  for (; i + 96 < len; i += 128) {  // four loads in flight per lane
+    const uint16_t a = src[i], b = src[i + 32], c = src[i + 64], d = src[i + 96];
+    dst[i] = a;
+    dst[i + 32] = b;
+    dst[i + 64] = c;
+    dst[i + 96] = d;
+  }
+  for (; i < len; i += 32) dst[i] = src[i];
 }
 
 }  // namespace
@@ -605,10 +738,13 @@ cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stre
   quant_kernel<<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, mode);
   if ((err = cudaGetLastError()) != cudaSuccess || build_only) return err;
   const uint64_t tiles = (p.C + kRThreads - 1) / kRThreads;
-  rans_kernel<<<unsigned(uint64_t(p.num_chunks) * p.L * 2 * tiles), kRThreads, 0, stream>>>(
-      p, mode == kModeSuppliedTables);
+  const unsigned rblocks = unsigned(uint64_t(p.num_chunks) * p.L * 2 * tiles);
+  if (mode == kModeSuppliedTables)
+    rans_kernel<true><<<rblocks, kRThreads, 0, stream>>>(p);
+  else
+    rans_kernel<false><<<rblocks, kRThreads, 0, stream>>>(p);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  scan_kernel<<<p.num_chunks, kScanThreads, 0, stream>>>(p);
+  offsets_kernel<<<unsigned(uint64_t(p.num_chunks) * p.L * 2), kScanThreads, 0, stream>>>(p);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const uint64_t streams = uint64_t(p.num_chunks) * p.L * 2 * p.C;
   compact_kernel<<<unsigned((streams + 7) / 8), 256, 0, stream>>>(p);

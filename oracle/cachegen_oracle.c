@@ -48,7 +48,7 @@ enum {
 
 #define ORC_GROUP 10
 #define ORC_M 4096u           /* 2^12: total of every frequency table */
-#define ORC_RANS_L 65536u     /* 2^16: lower bound of the rANS state */
+#define ORC_RANS_L 32768u     /* 2^15: lower bound of the rANS state */
 #define ORC_HEADER 64u
 #define ORC_MAGIC 0x314B4743u /* "CGK1" little-endian */
 
@@ -219,7 +219,8 @@ static int64_t rans_encode_tabs(const uint8_t* sym, int nsym, int per_table, con
     uint32_t fs = freq[(size_t)k * 256 + sym[j]];
     uint32_t cum = cums[(size_t)k * 257 + sym[j]];
     if (fs == 0) return -2;
-    if ((uint64_t)x >= ((uint64_t)fs << 20)) { /* renormalise: push 16 bits out */
+    /* renormalise: push 16 bits out when the step would leave [L, 2^16 L) */
+    if ((uint64_t)x >= (((uint64_t)ORC_RANS_L >> 12) << 16) * fs) {
       tmp[m++] = (uint16_t)(x & 0xFFFF);
       x >>= 16;
     }

@@ -17,32 +17,35 @@ def _table(fs):
 
 
 def test_hand_worked_one_symbol_stream(oracle_lib):
-    # f = {0: 4095, 1: 1}; encode [1] from x = 2^16: no renormalisation (65536 < 1 << 20),
-    # x = 65536 * 4096 + 0 + 4095 = 0x10000FFF -> words [0x1000, 0x0FFF].
+    # f = {0: 4095, 1: 1}; encode [1] from x = 2^15: no renormalisation (32768 < 1 << 19),
+    # x = 32768 * 4096 + 0 + 4095 = 0x08000FFF -> words [0x0800, 0x0FFF].
     f = _table({0: 4095, 1: 1})
     w = oracle_lib.rans_encode(np.array([1], np.uint8), 1, f)
-    assert w.tolist() == [0x1000, 0x0FFF]
+    assert w.tolist() == [0x0800, 0x0FFF]
     rc, s = oracle_lib.rans_decode(w, 1, 1, f)
     assert rc == 0 and s.tolist() == [1]
 
 
 def test_hand_worked_two_symbol_stream(oracle_lib):
-    # encode [0, 0] with f0 = 4095: 65536 -> 16*4096 + 16 = 65552 -> 16*4096 + 32 = 65568.
+    # encode [0, 0] with f0 = 4095: 32768 = 8*4095 + 8 -> 8*4096 + 8 = 32776
+    # = 8*4095 + 16 -> 8*4096 + 16 = 32784 = 0x8010 -> words [0x0000, 0x8010].
     f = _table({0: 4095, 1: 1})
     w = oracle_lib.rans_encode(np.array([0, 0], np.uint8), 2, f)
-    assert w.tolist() == [0x0001, 0x0020]
+    assert w.tolist() == [0x0000, 0x8010]
+    rc, s = oracle_lib.rans_decode(w, 2, 2, f)
+    assert rc == 0 and s.tolist() == [0, 0]
 
 
 def test_single_symbol_table_costs_only_the_state(oracle_lib):
     f = _table({42: 4096})
     w = oracle_lib.rans_encode(np.full(4096, 42, np.uint8), 4096, f)
-    assert w.tolist() == [1, 0]  # the state never moves from 2^16
+    assert w.tolist() == [0, 0x8000]  # the state never moves from 2^15
 
 
 @pytest.mark.parametrize("N", [1, 3, 4, 5, 8, 1023, 1024, 4096])
 def test_uniform_sixteen_symbol_closed_form(oracle_lib, N):
-    # 16 symbols at f = 256: each step multiplies the state by 16, so from 2^16 the
-    # state reaches 2^28 = 256 << 20 after three symbols and renormalises before every
+    # 16 symbols at f = 256: each step multiplies the state by 16, so from 2^15 the
+    # state reaches 2^27 = 256 << 19 after three symbols and renormalises before every
     # fourth: floor(N/4) words plus the two words of the final state.
     f = _table({u: 256 for u in range(16)})
     rng = np.random.default_rng(N)
