@@ -30,9 +30,7 @@ namespace cg {
 namespace {
 
 constexpr int kQThreads = 256;
-constexpr int kSlots = 3;                          // token slots in flight per thread (6 x 16 B)
-constexpr int kTileGroups = 16;
-constexpr int kTileTokens = kTileGroups * kGroup;  // 160
+constexpr int kQWarps = kQThreads / 32;
 constexpr int kRThreads = 128;                     // rANS streams per CTA
 constexpr int kRing = 64;                          // u16 ring entries per thread
 constexpr int kRingStride = 72;                    // u16; 144 B keeps 16-B alignment and
@@ -46,46 +44,42 @@ struct QSmem {
   uint32_t zp;      // f32 [256]
   uint32_t sc;      // f32 [256]
   uint32_t rcp;     // f32 [256]
-  uint32_t ahat;    // f32 [16][D + 4]  (phase B)
-  uint32_t red;     // f32 [2][512]     range reduction (phase A, aliases ahat)
-  uint32_t counts;  // u32 [256]        histogram totals (phase C, aliases ahat)
+  uint32_t red;     // f32 [2][8 warps][256]  anchor range partials (phase A)
+  uint32_t counts;  // u32 [256]  histogram totals (phase C, aliases red)
   uint32_t total;
 };
 
 __host__ __device__ inline uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
 
-__host__ __device__ inline QSmem q_smem(int D) {
+__host__ __device__ inline QSmem q_smem() {
   QSmem s;
   s.hist = 0;
   s.zp = a16(s.hist + 255u * 32u * 4u);
   s.sc = s.zp + 1024u;
   s.rcp = s.sc + 1024u;
-  s.ahat = s.rcp + 1024u;
-  // red (phase A) and counts (phase C) reuse the anchor buffer of phase B
-  s.red = s.ahat;
-  s.counts = s.ahat;
-  const uint32_t ahat_bytes = uint32_t(kTileGroups) * uint32_t(D + 4) * 4u;
-  const uint32_t red_bytes = 2u * 512u * 4u;
-  s.total = a16(s.ahat + (ahat_bytes > red_bytes ? ahat_bytes : red_bytes));
+  s.red = s.rcp + 1024u;
+  s.counts = s.red;
+  s.total = a16(s.red + 2u * kQWarps * 256u * 4u);
   return s;
 }
 
-// Exact quantisation of d = x - a by a step s with precomputed r = RN(1/s):
-// y = RN(d * r) differs from RN(d / s) by under 2^-21 |y|, so when y is
-// further than that from every half-integer both round to the same integer.
-// The integer is read from the bits of yc + (1.5 * 2^23 + 127): the low byte
-// is u = q + 127.  `ok` turns false when the shortcut cannot decide (a value
-// near a half-integer, a huge |y|, or a non-finite input).
+// Exact quantisation of d = x - a by a step s with precomputed r = RN(1/s).
+// y = RN(d * r) is within 3 * 2^-24 |y| of RN(d / s) (three roundings of
+// relative size 2^-24).  The two values yc (1 - 2^-20) and yc (1 + 2^-20), yc
+// = y clamped to [-127, 127], bracket RN(d / s) (clamped alike) with room to
+// spare; each is rounded to an integer by one fused add of 1.5 * 2^23 + 127
+// (ulp 1 there).  When both give the same integer, no half-integer lies
+// between them, so round-half-away-from-zero of RN(d / s) gives that integer
+// too, and the low byte of the sum is u = q + 127.  `ok` turns false when the
+// two differ (a value near a half-integer) or |y| >= 2^22 (a huge or
+// non-finite input); the caller then takes the definition itself.
 __device__ __forceinline__ uint32_t quant_fast(float d, float r, bool& ok) {
   const float y = __fmul_rn(d, r);
   const float yc = fminf(fmaxf(y, -127.0f), 127.0f);
-  const float t = __fadd_rn(yc, 12583039.0f);
-  const float k = __fsub_rn(t, 12583039.0f);
-  const float e = __fsub_rn(yc, k);
-  const float gap = __fsub_rn(0.5f, fabsf(e));
-  const float m = __fmaf_rn(fabsf(y), -0x1p-21f, gap);  // exact sign of gap - |y| 2^-21
-  ok = ok && (m > 0.0f);
-  return __float_as_uint(t) & 0xFFu;
+  const float t1 = __fmaf_rn(yc, 1.0f + 0x1p-20f, 12583039.0f);
+  const float t2 = __fmaf_rn(yc, 1.0f - 0x1p-20f, 12583039.0f);
+  ok = ok && (__float_as_uint(t1) == __float_as_uint(t2)) && (fabsf(y) < 0x1p22f);
+  return __float_as_uint(t1) & 0xFFu;
 }
 
 // The definition itself: u = clamp(roundf(RN(RN(x - a) / s)), -127, 127) + 127,
@@ -209,7 +203,36 @@ __device__ __forceinline__ uint4 enc_entry(uint32_t f, uint32_t cum) {
   return make_uint4((f << 19) - 1u, magic, cum, ((kM - f) << 5) | lg);
 }
 
-__global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const EncParams p, const int mode) {
+// Lane layout of the quantiser: a lane covers 8 channels (one 16-byte load of
+// a token's head row); D/8 lanes cover a row, so a warp covers rpw = 32/(D/8)
+// rows at once and works on rpw anchor groups side by side (lane row r takes
+// group gs * rpw + r of group set gs).
+struct QLanes {
+  int lpr, rpw, r, c;
+  bool on;
+};
+
+__device__ __forceinline__ QLanes q_lanes(int D, int lane) {
+  QLanes q;
+  q.lpr = D / 8;
+  q.rpw = 32 / q.lpr;
+  q.r = lane / q.lpr;
+  q.c = lane - q.r * q.lpr;
+  q.on = q.r < q.rpw;
+  return q;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 rv, float (&x)[8]) {
+  const uint32_t raw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q]));
+    x[2 * q] = f2.x;
+    x[2 * q + 1] = f2.y;
+  }
+}
+
+__global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, const int mode) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int rest = blockIdx.x;
@@ -228,15 +251,13 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const EncParams p, 
   const uint64_t rs = uint64_t(H) * D;
   const uint16_t* col = p.kv + (uint64_t(slab) * p.T + t0) * rs + uint64_t(h) * D;
 
-  const QSmem sm = q_smem(D);
+  const QSmem sm = q_smem();
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + sm.hist);
   float* zp = reinterpret_cast<float*>(smem + sm.zp);
   float* sc = reinterpret_cast<float*>(smem + sm.sc);
   float* rcp = reinterpret_cast<float*>(smem + sm.rcp);
-  float* ahat = reinterpret_cast<float*>(smem + sm.ahat);
   float* red = reinterpret_cast<float*>(smem + sm.red);
   uint32_t* counts = reinterpret_cast<uint32_t*>(smem + sm.counts);
-  const int astride = D + 4;
 
   const Sections sec = sections(L, H, D, n);
   uint8_t* cont = p.out ? p.out + uint64_t(chunk) * p.out_stride : nullptr;
@@ -245,6 +266,9 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const EncParams p, 
                  tb_fq = sec.freq - CG_HEADER_BYTES;
   const bool want_hist = mode != kModeSuppliedTables;
   const bool want_sym = mode != kModeTablesOnly;
+  const QLanes ql = q_lanes(D, lane);
+  const int ch = 8 * ql.c;  // first channel of this lane
+  const int nsets = (Gn + ql.rpw - 1) / ql.rpw;
 
   if (want_hist)
     for (int i = tid; i < kAlphabet * 32; i += kQThreads) hist[i] = 0;
@@ -259,45 +283,53 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const EncParams p, 
       sc[d] = reinterpret_cast<const float*>(tb + tb_sc)[uint64_t(tab) * D + d];
     }
   } else {
-    const int np = D / 2;             // fp16 pairs per row
-    const int rp = kQThreads / np;    // anchor rows scanned in parallel (>= 2)
-    const int pi = tid % np, r = tid / np;
-    float lo0 = __int_as_float(0x7F800000), hi0 = -lo0, lo1 = lo0, hi1 = hi0;
-    if (r < rp) {
-      for (int g0 = r; g0 < Gn; g0 += 8 * rp) {  // eight anchor rows in flight
-        uint32_t v[8];
+    float lo[8], hi[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int g = g0 + j * rp;
-          v[j] = g < Gn ? __ldg(reinterpret_cast<const uint32_t*>(col + uint64_t(g) * kGroup * rs) + pi)
-                        : 0u;
-        }
+    for (int k = 0; k < 8; ++k) {
+      lo[k] = __int_as_float(0x7F800000);
+      hi[k] = -lo[k];
+    }
+    for (int gs = warp; gs < nsets; gs += 4 * kQWarps) {  // four anchor rows in flight
+      uint4 v[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (g0 + j * rp >= Gn) continue;
-          const float a = half_bits_to_float(uint16_t(v[j] & 0xFFFF));
-          const float b = half_bits_to_float(uint16_t(v[j] >> 16));
-          if (!isfinite(a) || !isfinite(b)) nonfinite = true;
-          lo0 = fminf(lo0, a);
-          hi0 = fmaxf(hi0, a);
-          lo1 = fminf(lo1, b);
-          hi1 = fmaxf(hi1, b);
+      for (int j = 0; j < 4; ++j) {
+        const int g = (gs + j * kQWarps) * ql.rpw + ql.r;
+        v[j] = ql.on && g < Gn
+                   ? __ldg(reinterpret_cast<const uint4*>(col + uint64_t(g) * kGroup * rs + ch))
+                   : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int g = (gs + j * kQWarps) * ql.rpw + ql.r;
+        if (!(ql.on && g < Gn)) continue;
+        float x[8];
+        unpack8(v[j], x);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (!isfinite(x[k])) nonfinite = true;
+          lo[k] = fminf(lo[k], x[k]);
+          hi[k] = fmaxf(hi[k], x[k]);
         }
       }
-      red[r * D + 2 * pi] = lo0;
-      red[r * D + 2 * pi + 1] = lo1;
-      red[512 + r * D + 2 * pi] = hi0;
-      red[512 + r * D + 2 * pi + 1] = hi1;
+    }
+    // partials of (warp, lane row) -> red[{lo, hi}][warp * rpw + r][channel]
+    if (ql.on) {
+      float* rl = red + (warp * ql.rpw + ql.r) * D + ch;
+      float* rh = rl + kQWarps * 256;
+      *reinterpret_cast<float4*>(rl) = make_float4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<float4*>(rl + 4) = make_float4(lo[4], lo[5], lo[6], lo[7]);
+      *reinterpret_cast<float4*>(rh) = make_float4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<float4*>(rh + 4) = make_float4(hi[4], hi[5], hi[6], hi[7]);
     }
     __syncthreads();
     for (int d = tid; d < D; d += kQThreads) {
-      float lo = red[d], hi = red[512 + d];
-      for (int j = 1; j < rp; ++j) {
-        lo = fminf(lo, red[j * D + d]);
-        hi = fmaxf(hi, red[512 + j * D + d]);
+      float lo1 = red[d], hi1 = red[kQWarps * 256 + d];
+      for (int j = 1; j < kQWarps * ql.rpw; ++j) {
+        lo1 = fminf(lo1, red[j * D + d]);
+        hi1 = fmaxf(hi1, red[kQWarps * 256 + j * D + d]);
       }
-      zp[d] = __fmul_rn(__fadd_rn(lo, hi), 0.5f);
-      sc[d] = __fdiv_rn(__fsub_rn(hi, lo), 254.0f);
+      zp[d] = __fmul_rn(__fadd_rn(lo1, hi1), 0.5f);
+      sc[d] = __fdiv_rn(__fsub_rn(hi1, lo1), 254.0f);
     }
   }
   __syncthreads();
@@ -315,122 +347,92 @@ __global__ void __launch_bounds__(kQThreads, 3) quant_kernel(const EncParams p, 
   }
   __syncthreads();
 
-  // ---- Phase B: quantise the chunk tile by tile (16 groups per tile).
+  // ---- Phase B: quantise group by group.  Each lane loads the ten rows of its
+  // group for its 8 channels; the rows of the warp's next group set are loaded
+  // before the current set is quantised.
   const float step = step_of(p.level, l, L);
   const float rstep = __frcp_rn(step);
-  const int nb = D / 16;            // 16-value blocks per row
-  const int tpw = 32 / nb;          // tokens per warp and pass
-  const int tw = lane / nb, b = lane % nb;
-  const bool lane_ok = lane < tpw * nb;
-  uint8_t* symc = p.sym + ((uint64_t(chunk) * L * 2 + slab) * H + h) * uint64_t(nb) * C * 16;
-
-  for (int tb = 0; tb < n; tb += kTileTokens) {
-    const int g0 = tb / kGroup;
-    const int ng = min(kTileGroups, Gn - g0);
-    // B1: anchor codes and reconstructed anchors of the tile's groups, eight
-    // channels (one 16-byte load) per thread.
-    for (int idx = tid; idx < ng * (D / 8); idx += kQThreads) {
-      const int gi = idx / (D / 8), d = (idx - gi * (D / 8)) * 8;
-      const int t = tb + kGroup * gi;
-      const uint4 rv = __ldg(reinterpret_cast<const uint4*>(col + uint64_t(t) * rs + d));
-      const uint32_t raw[4] = {rv.x, rv.y, rv.z, rv.w};
-      uint32_t u[8];
-      float av[8];
+  uint8_t* symc = p.sym + ((uint64_t(chunk) * L * 2 + slab) * H + h) * uint64_t(D / 16) * C * 16 +
+                  (ql.c >> 1) * uint64_t(C) * 16 + (ql.c & 1) * 8;
+  uint4 nx[kGroup];
+  auto load_set = [&](int gs, uint4 (&v)[kGroup]) {
+    const int g = gs * ql.rpw + ql.r;
+    const int tg = g * kGroup;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q]));
-        const float xs[2] = {f2.x, f2.y};
+    for (int j = 0; j < kGroup; ++j)
+      v[j] = ql.on && gs < nsets && g < Gn && tg + j < n
+                 ? __ldg(reinterpret_cast<const uint4*>(col + uint64_t(tg + j) * rs + ch))
+                 : make_uint4(0, 0, 0, 0);
+  };
+  load_set(warp, nx);
+  for (int gs = warp; gs < nsets; gs += kQWarps) {
+    uint4 cur[kGroup];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int dd = d + 2 * q + e;
-          const float x = xs[e];
-          if (!isfinite(x)) nonfinite = true;
-          bool ok = true;
-          uint32_t uu = quant_fast(__fsub_rn(x, zp[dd]), rcp[dd], ok);
-          if (!ok) uu = quant_exact(x, zp[dd], sc[dd]);
-          u[2 * q + e] = uu;
-          av[2 * q + e] = __fadd_rn(zp[dd], __fmul_rn(float(int(uu) - 127), sc[dd]));
-        }
+    for (int j = 0; j < kGroup; ++j) cur[j] = nx[j];
+    load_set(gs + kQWarps, nx);
+    const int g = gs * ql.rpw + ql.r;
+    if (!(ql.on && g < Gn)) continue;
+    const int tg = g * kGroup;
+    const int ntok = min(kGroup, n - tg);
+    // anchor: code against (zp, scale), reconstructed value a
+    float a[8];
+    {
+      float x[8], zc[8], scc[8], rc[8];
+      unpack8(cur[0], x);
+#pragma unroll
+      for (int k = 0; k < 8; k += 4) {  // this lane's channels, from shared memory
+        const float4 za = *reinterpret_cast<const float4*>(zp + ch + k);
+        const float4 sa = *reinterpret_cast<const float4*>(sc + ch + k);
+        const float4 ra = *reinterpret_cast<const float4*>(rcp + ch + k);
+        zc[k] = za.x; zc[k + 1] = za.y; zc[k + 2] = za.z; zc[k + 3] = za.w;
+        scc[k] = sa.x; scc[k + 1] = sa.y; scc[k + 2] = sa.z; scc[k + 3] = sa.w;
+        rc[k] = ra.x; rc[k + 1] = ra.y; rc[k + 2] = ra.z; rc[k + 3] = ra.w;
       }
-      *reinterpret_cast<float4*>(ahat + gi * astride + d) = make_float4(av[0], av[1], av[2], av[3]);
-      *reinterpret_cast<float4*>(ahat + gi * astride + d + 4) =
-          make_float4(av[4], av[5], av[6], av[7]);
+      uint32_t u[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (!isfinite(x[k])) nonfinite = true;
+        bool ok = true;
+        u[k] = quant_fast(__fsub_rn(x[k], zc[k]), rc[k], ok);
+        if (!ok) u[k] = quant_exact(x[k], zc[k], scc[k]);
+        a[k] = __fadd_rn(zc[k], __fmul_rn(float(int(u[k]) - 127), scc[k]));
+      }
       if (want_hist) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) atomicAdd(&hist[u[q] * 32 + lane], 1u);
+        for (int k = 0; k < 8; ++k) atomicAdd(&hist[u[k] * 32 + lane], 1u);
       }
       if (want_sym)
-        *reinterpret_cast<uint2*>(symc + (uint64_t(d >> 4) * C + t) * 16 + (d & 15)) =
+        *reinterpret_cast<uint2*>(symc + uint64_t(tg) * 16) =
             make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
                        u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
     }
-    __syncthreads();
-    // B2: the delta tokens of the tile; lane -> (token slot, 16-value block),
-    // kSlots token slots per pass so that 2 * kSlots 16-byte loads are in flight.
-    if (lane_ok) {
-      const int kslots = ng * (kGroup - 1);
-      const int kstride = (kQThreads / 32) * tpw;
-      for (int k = warp * tpw + tw; k < kslots; k += kSlots * kstride) {
-        int gi[kSlots], tk[kSlots];
-        bool has[kSlots];
-        uint4 r[kSlots][2];
 #pragma unroll
-        for (int j = 0; j < kSlots; ++j) {
-          const int kk = k + j * kstride;
-          gi[j] = kk / (kGroup - 1);
-          tk[j] = tb + kGroup * gi[j] + 1 + (kk - gi[j] * (kGroup - 1));
-          has[j] = kk < kslots && tk[j] < n;
-          if (has[j]) {
-            const uint4* src = reinterpret_cast<const uint4*>(col + uint64_t(tk[j]) * rs + 16 * b);
-            r[j][0] = __ldg(src);
-            r[j][1] = __ldg(src + 1);
-          }
-        }
+    for (int j = 1; j < kGroup; ++j) {
+      if (j >= ntok) break;
+      float x[8];
+      unpack8(cur[j], x);
+      bool ok = true;
+      uint32_t u[8];
 #pragma unroll
-        for (int j = 0; j < kSlots; ++j) {
-          if (!has[j]) continue;
-          const float* arow = ahat + gi[j] * astride + 16 * b;
-          uint32_t pk[4];
+      for (int k = 0; k < 8; ++k) u[k] = quant_fast(__fsub_rn(x[k], a[k]), rstep, ok);
+      if (!ok) {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {  // 8 values at a time keeps registers low
-            const uint4 rv = r[j][half];
-            const uint32_t raw[4] = {rv.x, rv.y, rv.z, rv.w};
-            const float4 av0 = *reinterpret_cast<const float4*>(arow + 8 * half);
-            const float4 av1 = *reinterpret_cast<const float4*>(arow + 8 * half + 4);
-            const float a[8] = {av0.x, av0.y, av0.z, av0.w, av1.x, av1.y, av1.z, av1.w};
-            float x[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&raw[q]));
-              x[2 * q] = f2.x;
-              x[2 * q + 1] = f2.y;
-            }
-            bool ok = true;
-            uint32_t u[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) u[q] = quant_fast(__fsub_rn(x[q], a[q]), rstep, ok);
-            if (!ok) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                if (!isfinite(x[q])) nonfinite = true;
-                u[q] = quant_exact(x[q], a[q], step);
-              }
-            }
-            if (want_hist) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) atomicAdd(&hist[u[q] * 32 + lane], 1u);
-            }
-            pk[2 * half] = u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24);
-            pk[2 * half + 1] = u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24);
-          }
-          if (want_sym)
-            *reinterpret_cast<uint4*>(symc + (uint64_t(b) * C + tk[j]) * 16) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int k = 0; k < 8; ++k) {
+          if (!isfinite(x[k])) nonfinite = true;
+          u[k] = quant_exact(x[k], a[k], step);
         }
       }
+      if (want_hist) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) atomicAdd(&hist[u[k] * 32 + lane], 1u);
+      }
+      if (want_sym)
+        *reinterpret_cast<uint2*>(symc + uint64_t(tg + j) * 16) =
+            make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
+                       u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
     }
-    __syncthreads();
   }
+  __syncthreads();
   if (nonfinite) set_status(p.status, CG_ERR_NONFINITE);
 
   // ---- Phase C: histogram -> frequency table -> encoder constants.
@@ -545,7 +547,9 @@ __global__ void __launch_bounds__(kRThreads, 6) rans_kernel(const EncParams p) {
   uint32_t x = kRansL, wp = 0, wf = 0;
   bool bad = false;
   int blk = H * nb - 1;  // next 16-symbol block, walking backwards
+  // symbol blocks are loaded two blocks (32 symbols) ahead of their use
   uint4 vnext = active ? __ldg(symt + uint64_t(blk) * C) : make_uint4(0, 0, 0, 0);
+  uint4 vnext2 = active && blk > 0 ? __ldg(symt + uint64_t(blk - 1) * C) : make_uint4(0, 0, 0, 0);
   for (int h = H - 1; h >= 0; --h) {
     uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
     if (h > 0) {
@@ -557,7 +561,8 @@ __global__ void __launch_bounds__(kRThreads, 6) rans_kernel(const EncParams p) {
     if (active) {
       for (int b = nb - 1; b >= 0; --b, --blk) {
         const uint4 v = vnext;
-        if (blk > 0) vnext = __ldg(symt + uint64_t(blk - 1) * C);
+        vnext = vnext2;
+        if (blk > 1) vnext2 = __ldg(symt + uint64_t(blk - 2) * C);
 #pragma unroll
         for (int k = 15; k >= 0; --k) {
           const uint32_t word = (k >> 2) == 0 ? v.x : (k >> 2) == 1 ? v.y : (k >> 2) == 2 ? v.z : v.w;
@@ -730,7 +735,7 @@ __global__ void __launch_bounds__(256) compact_kernel(const EncParams p) {
 cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stream) {
   const int mode =
       build_only ? kModeTablesOnly : (p.tables_in ? kModeSuppliedTables : kModeEncode);
-  const QSmem sm = q_smem(p.D);
+  const QSmem sm = q_smem();
   cudaError_t err = cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          int(sm.total));
   if (err != cudaSuccess) return err;
