@@ -719,15 +719,45 @@ __global__ void __launch_bounds__(256) compact_kernel(const EncParams p) {
   const uint16_t* src =
       reinterpret_cast<const uint16_t*>(p.scratch + (cs * C + t + 1) * scratch_stride(H, D)) - len;
   uint16_t* dst = reinterpret_cast<uint16_t*>(cont + sec.payload + o0);
-  uint32_t i = lane;
-  for (; i + 96 < len; i += 128) {  // four loads in flight per lane
-    const uint16_t a = src[i], b = src[i + 32], c = src[i + 64], d = src[i + 96];
-    dst[i] = a;
-    dst[i + 32] = b;
-    dst[i + 64] = c;
-    dst[i + 96] = d;
+  // The payload is written in 16-byte aligned chunks; the few u16 words before
+  // the first chunk and after the last one are copied one by one.  A chunk's
+  // source bytes start at an even offset o within an aligned 16-byte block, so
+  // each output word is a funnel shift of two adjacent source words.
+  const uint32_t nbytes = 2u * len;
+  const uint32_t head = uint32_t((16u - (reinterpret_cast<uintptr_t>(dst) & 15u)) & 15u);
+  if (nbytes < head + 16u) {
+    for (uint32_t i = lane; i < len; i += 32) dst[i] = src[i];
+    return;
   }
-  for (; i < len; i += 32) dst[i] = src[i];
+  const uint32_t nchunks = (nbytes - head) / 16u;
+  const uint32_t tail = (head + nchunks * 16u) / 2u;  // first word after the chunks
+  if (lane < head / 2u) dst[lane] = src[lane];
+  for (uint32_t i = tail + lane; i < len; i += 32) dst[i] = src[i];
+  const uint8_t* sm = reinterpret_cast<const uint8_t*>(src) + head;
+  const uint32_t o = uint32_t(reinterpret_cast<uintptr_t>(sm) & 15u);
+  const uint4* sa = reinterpret_cast<const uint4*>(sm - o);
+  uint4* dm = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dst) + head);
+  const uint32_t q = o >> 2, sh = 8u * (o & 3u);
+  for (uint32_t k = lane; k < nchunks; k += 32) {
+    const uint4 a = sa[k];
+    // the next block holds bytes of this chunk only when o != 0; it then ends
+    // at or before the end of the stream's slot
+    const uint4 b = o != 0 ? sa[k + 1] : make_uint4(0, 0, 0, 0);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo, hi;
+      switch (q) {  // warp-uniform
+        case 0: lo = w[i]; hi = w[i + 1]; break;
+        case 1: lo = w[i + 1]; hi = w[i + 2]; break;
+        case 2: lo = w[i + 2]; hi = w[i + 3]; break;
+        default: lo = w[i + 3]; hi = w[i + 4]; break;
+      }
+      r[i] = __funnelshift_r(lo, hi, sh);
+    }
+    dm[k] = make_uint4(r[0], r[1], r[2], r[3]);
+  }
 }
 
 }  // namespace
