@@ -32,6 +32,12 @@
 // round-to-nearest adds and multiplies (no contraction).  The slot entry keeps
 // the symbol in its top byte, so (float)q comes from a byte permute and one
 // exact subtraction instead of a second shared-memory lookup.
+//
+// Output: a thread's values of two steps (16 fp16, 32 contiguous bytes of its
+// token's row) leave as one 256-bit store, a full L2 sector.  Every thread
+// writes its own row, so a warp's store touches 32 rows; with 16-byte stores
+// the L2 had to take twice as many partial-sector writes, which bounded the
+// kernel more than the decoding itself.
 #include <cuda_fp16.h>
 
 #include "cg_common.cuh"
@@ -251,29 +257,48 @@ struct Pos {
   uint32_t p, ra, w;
 };
 
-// Delta lane: decode head h of its stream in steps of 8 values.
+// 32-byte store of 16 fp16 values (one full sector); two 16-byte stores when
+// the destination is only 16-byte aligned.
+__device__ __forceinline__ void store16h(uint16_t* dst, const uint32_t (&hv)[8], bool al32) {
+  if (al32) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"l"(dst),
+                 "r"(hv[0]), "r"(hv[1]), "r"(hv[2]), "r"(hv[3]), "r"(hv[4]), "r"(hv[5]),
+                 "r"(hv[6]), "r"(hv[7])
+                 : "memory");
+  } else {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    *reinterpret_cast<uint4*>(dst + 8) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
+  }
+}
+
+// Delta lane: decode head h of its stream in steps of 8 values; the values of
+// two steps leave as one 32-byte store.
 __device__ __forceinline__ void decode_delta_head(uint32_t& x, Pos& ps, Ring& r,
                                                   const uint32_t* __restrict__ tbl, float step,
                                                   const float* __restrict__ arow,
-                                                  uint16_t* __restrict__ orow, int D) {
-  for (int d0 = 0; d0 < D; d0 += 8) {
-    ring_issue(r, ps.p);
-    ring_wait_two_steps();
-    const uint32_t ra0 = ps.ra;
-    const float4 a0 = *reinterpret_cast<const float4*>(arow + d0);
-    const float4 a1 = *reinterpret_cast<const float4*>(arow + d0 + 4);
-    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    uint32_t hv[4];
+                                                  uint16_t* __restrict__ orow, int D, bool al32) {
+  for (int d0 = 0; d0 < D; d0 += 16) {
+    uint32_t hv[8];
 #pragma unroll
-    for (int k = 0; k < 8; k += 2) {
-      const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
-      const float v0 = __fadd_rn(a[k], __fmul_rn(sym_value(e0), step));
-      const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
-      const float v1 = __fadd_rn(a[k + 1], __fmul_rn(sym_value(e1), step));
-      hv[k >> 1] = pack_half2(v0, v1);
+    for (int half = 0; half < 2; ++half) {
+      const int dd = d0 + 8 * half;
+      ring_issue(r, ps.p);
+      ring_wait_two_steps();
+      const uint32_t ra0 = ps.ra;
+      const float4 a0 = *reinterpret_cast<const float4*>(arow + dd);
+      const float4 a1 = *reinterpret_cast<const float4*>(arow + dd + 4);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int k = 0; k < 8; k += 2) {
+        const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+        const float v0 = __fadd_rn(a[k], __fmul_rn(sym_value(e0), step));
+        const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+        const float v1 = __fadd_rn(a[k + 1], __fmul_rn(sym_value(e1), step));
+        hv[4 * half + (k >> 1)] = pack_half2(v0, v1);
+      }
+      ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
     }
-    ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
-    *reinterpret_cast<uint4*>(orow + d0) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    store16h(orow + d0, hv, al32);
   }
 }
 
@@ -284,29 +309,34 @@ __device__ __forceinline__ void decode_anchor_head(uint32_t& x, Pos& ps, Ring& r
                                                    const float* __restrict__ zp,
                                                    const float* __restrict__ sc,
                                                    float* __restrict__ arow,
-                                                   uint16_t* __restrict__ orow, int D) {
-  for (int d0 = 0; d0 < D; d0 += 8) {
-    ring_issue(r, ps.p);
-    ring_wait_two_steps();
-    const uint32_t ra0 = ps.ra;
-    const float4 z0 = *reinterpret_cast<const float4*>(zp + d0);
-    const float4 z1 = *reinterpret_cast<const float4*>(zp + d0 + 4);
-    const float4 s0 = *reinterpret_cast<const float4*>(sc + d0);
-    const float4 s1 = *reinterpret_cast<const float4*>(sc + d0 + 4);
-    const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-    const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-    float v[8];
+                                                   uint16_t* __restrict__ orow, int D, bool al32) {
+  for (int d0 = 0; d0 < D; d0 += 16) {
+    uint32_t hv[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t e = rans_step(x, ps.ra, ps.w, tbl, r.rb);
-      v[k] = __fadd_rn(z[k], __fmul_rn(sym_value(e), s[k]));
+    for (int half = 0; half < 2; ++half) {
+      const int dd = d0 + 8 * half;
+      ring_issue(r, ps.p);
+      ring_wait_two_steps();
+      const uint32_t ra0 = ps.ra;
+      const float4 z0 = *reinterpret_cast<const float4*>(zp + dd);
+      const float4 z1 = *reinterpret_cast<const float4*>(zp + dd + 4);
+      const float4 s0 = *reinterpret_cast<const float4*>(sc + dd);
+      const float4 s1 = *reinterpret_cast<const float4*>(sc + dd + 4);
+      const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+      const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      float v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t e = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+        v[k] = __fadd_rn(z[k], __fmul_rn(sym_value(e), s[k]));
+      }
+      ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
+      *reinterpret_cast<float4*>(arow + dd) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(arow + dd + 4) = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) hv[4 * half + k] = pack_half2(v[2 * k], v[2 * k + 1]);
     }
-    ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
-    *reinterpret_cast<float4*>(arow + d0) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4*>(arow + d0 + 4) = make_float4(v[4], v[5], v[6], v[7]);
-    *reinterpret_cast<uint4*>(orow + d0) =
-        make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]), pack_half2(v[4], v[5]),
-                   pack_half2(v[6], v[7]));
+    store16h(orow + d0, hv, al32);
   }
 }
 
@@ -398,6 +428,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
     }
   }
   const float step = step_of(p.level, l, L);
+  // 32-byte stores need a 32-byte aligned destination (rows are multiples of 32 bytes)
+  const bool al32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
   __syncthreads();
   if (s_bad) {
     if (tid == 0) set_status(p.status, CG_ERR_CORRUPT);
@@ -504,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
                            pack_half2(v[4], v[5]), pack_half2(v[6], v[7]));
           }
         } else {
-          decode_anchor_head(x, ps, ring, tb, zh, zh + D, arow, orow + h * D, D);
+          decode_anchor_head(x, ps, ring, tb, zh, zh + D, arow, orow + h * D, D, al32);
         }
       }
     } else if (it >= 1 && active) {
@@ -522,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
           *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
       } else {
-        decode_delta_head(x, ps, ring, tb, step, arow, orow + h * D, D);
+        decode_delta_head(x, ps, ring, tb, step, arow, orow + h * D, D, al32);
       }
     }
     if (scan_warp) cum_compact(fq, cum_buf(cumb + (it & 1) * kCumBuf), lane);

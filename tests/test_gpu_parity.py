@@ -78,6 +78,11 @@ RAGGED = [  # L, H, D, T, C
     (3, 2, 64, 300, 300),
     (2, 1, 16, 1000, 512),
     (4, 5, 80, 333, 100),
+    # the implementation's maxima: chunk of 16,384 tokens; 1,024 layers;
+    # 64 heads x head_dim 256 (streams of 16,384 symbols)
+    (1, 1, 16, 16384, 16384),
+    (1024, 1, 16, 12, 12),
+    (1, 64, 256, 12, 12),
 ]
 
 
@@ -137,3 +142,34 @@ def test_capacity_status():
     torch.cuda.synchronize()
     assert int(enc.sizes[0]) == int(full.sizes[0])  # the required size is reported
     del shape
+
+
+def test_destination_only_16_byte_aligned():
+    # The decoder writes 32-byte pieces when the destination allows it and
+    # 16-byte pieces otherwise; both must give the same bytes.
+    L, H, D, T, C = 3, 2, 64, 250, 96
+    kv = gu.gen(L, H, D, T, seed=11)
+    shape = Shape(L, H, D)
+    nch = -(-T // C)
+    enc = ta.encode(kv, C, 1)
+    ref, st = ta.decode(enc.data, enc.stride, shape, C, 1, nch)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == 0
+    flat = torch.empty(ref.numel() + 8, dtype=torch.int16, device=kv.device)
+    out = flat[8:]
+    assert out.data_ptr() % 32 == 16
+    out, st = ta.decode(enc.data, enc.stride, shape, C, 1, nch, out=out)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == 0
+    for k in range(nch):  # the written part of each chunk slot
+        n = min(C, T - k * C)
+        assert torch.equal(gu.chunk_slot(out, shape, C, k, n), gu.chunk_slot(ref, shape, C, k, n))
+    flat2 = torch.full((kv.numel() + 8,), 0x7E00, dtype=torch.int16, device=kv.device)
+    kv2 = flat2[8:].view(kv.shape)
+    assert kv2.data_ptr() % 32 == 16
+    st = ta.decode_into(enc.data, enc.stride, shape, C, 1, nch, kv2)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == 0
+    for k in range(nch):
+        n = min(C, T - k * C)
+        assert torch.equal(kv2[:, :, k * C:k * C + n], gu.chunk_slot(ref, shape, C, k, n))
