@@ -576,9 +576,12 @@ __global__ void __launch_bounds__(kRThreads, 6) rans_kernel(const EncParams p) {
         if (wp - wf >= 16) {
           const uint4* src = reinterpret_cast<const uint4*>(myring + (wf & (kRing - 1)));
           const uint4 r0 = src[0], r1 = src[1];
-          uint4* dst = reinterpret_cast<uint4*>(rend - wf - 16);
-          dst[0] = make_uint4(swap16(r1.w), swap16(r1.z), swap16(r1.y), swap16(r1.x));
-          dst[1] = make_uint4(swap16(r0.w), swap16(r0.z), swap16(r0.y), swap16(r0.x));
+          // one 256-bit store (a full L2 sector; rend - wf - 16 is 32-byte aligned)
+          uint16_t* dst = rend - wf - 16;
+          asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"l"(dst),
+                       "r"(swap16(r1.w)), "r"(swap16(r1.z)), "r"(swap16(r1.y)), "r"(swap16(r1.x)),
+                       "r"(swap16(r0.w)), "r"(swap16(r0.z)), "r"(swap16(r0.y)), "r"(swap16(r0.x))
+                       : "memory");
           wf += 16;
         }
       }
