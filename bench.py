@@ -33,6 +33,12 @@ WORKLOAD = dict(name="llama2_7b", L=32, H=32, D=128, T=10752, C=1536, seed=2, rh
                 p_out=0.01, m_out=8.0, level=1)
 METRIC = "cg_decode / cg_encode GB/s (fp16 KV) on 1 B200, % of HBM roofline, compression ratio"
 FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes (read + write) per fp16 value of decode_kernel from one ncu capture
+# of the current kernel (profiles/decode_kernel_mistral7b_3072tok.md: 103.9 MB
+# read + 350.4 MB written for 32x2x3072x8x128 = 201,326,592 values); the bench
+# reports it scaled by its own value count.  The capture ends with up to one L2
+# (126 MB) of written lines not yet in DRAM, so this slightly undercounts.
+DECODE_DRAM_BYTES_PER_VALUE = (103_941_888 + 350_364_160) / 201_326_592
 
 
 def _peaks():
@@ -283,7 +289,10 @@ def run_ours(args):
             "roofline": {"kernel": "decode_kernel (cg_decode_into)", "bound": "hbm",
                          "achieved": round(alg / ms_dec / 1e6, 1), "peak": hbm,
                          "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s",
-                         "frac": round(dec_frac, 4), "traffic": None,
+                         "frac": round(dec_frac, 4),
+                         "traffic": int(DECODE_DRAM_BYTES_PER_VALUE * (fp16_bytes // 2)),
+                         "traffic_source": "ncu dram bytes per value of a 3,072-token "
+                                           "Mistral-7B-shaped capture, scaled by values",
                          "algorithmic_bytes": alg},
             "gpu_launches": 5 * args.steps,
             "clocks": clocks,
