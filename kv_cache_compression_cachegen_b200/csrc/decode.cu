@@ -21,7 +21,8 @@
 // one __syncthreads per head separates the iterations.
 //
 // Compressed words reach a thread through a 64-byte ring in shared memory
-// (four 16-byte blocks).  Every 8 symbols the thread issues at most one
+// (four 16-byte blocks, plus a copy of the first block after the last, so that
+// the reads of one step never wrap).  Every 8 symbols the thread issues at most one
 // cp.async for the next block of its stream and waits only for the blocks
 // issued two steps earlier; since 8 symbols consume at most 8 words (one
 // block), the words a step can read were always requested at least two steps
@@ -54,12 +55,13 @@ constexpr uint32_t kCumBuf = 800;                      // bytes per compacted-ta
 constexpr uint32_t kRingBytes = 64;                    // per thread: 4 blocks of 16 bytes
 constexpr uint32_t kRingBlocks = kRingBytes / 16;
 constexpr uint32_t kRingWords = kRingBytes / 2;
+constexpr uint32_t kRingStride = kRingBytes + 16;       // + a copy of slot 0 after slot 3
 
 // Dynamic shared memory layout (byte offsets), a function of H and D.
 struct DecSmem {
   uint32_t tbl;     // u32 [3][4096]  slot tables, packed (u << 24) | (f << 12) | (slot - cum)
   uint32_t ahat;    // f32 [2][32][D + 4]  reconstructed anchors of the last two heads
-  uint32_t ring;    // u8  [320][64]  per-thread word rings (64-byte aligned)
+  uint32_t ring;    // u8  [320][80]  per-thread word rings: 4 slots + a mirror of slot 0
   uint32_t cum;     // [2] x {u16 pcum[257], u8 psym[256], i32 nz}: the next two heads' present
                     //        symbols in order and their cumulative frequencies
   uint32_t zs;      // f32 [2][2][D]  zero points and scales of the anchor warp's next heads
@@ -73,10 +75,8 @@ __host__ __device__ inline DecSmem dec_smem(int H, int D) {
   DecSmem s;
   s.tbl = 0;
   s.ahat = al16(s.tbl + 3u * 4096u * 4u);
-  // the rings are realigned to 64 bytes in the absolute shared address space,
-  // hence the 64 bytes of slack
   s.ring = al16(s.ahat + 2u * kUnitGroups * uint32_t(D + 4) * 4u);
-  s.cum = al16(s.ring + uint32_t(kThreads) * kRingBytes + 64u);
+  s.cum = al16(s.ring + uint32_t(kThreads) * kRingStride);
   s.zs = al16(s.cum + 2u * kCumBuf);
   s.single = al16(s.zs + 4u * uint32_t(D) * 4u);
   s.total = al16(s.single + uint32_t(H) * 4u);
@@ -88,27 +88,33 @@ __host__ __device__ inline DecSmem dec_smem(int H, int D) {
 // offset 2 * (q mod 32): block b = q / 8 occupies slot b mod 4.
 struct Ring {
   const uint8_t* gbase;  // container start (16-byte aligned)
-  uint32_t rb;           // shared-memory address of this thread's ring (64-byte aligned)
+  uint32_t rb;           // shared-memory address of this thread's ring (16-byte aligned)
   uint32_t fb;           // next 16-byte block of the container to request
   uint32_t lim;          // number of 16-byte blocks in the container
 };
 
 // Request the next block if the ring has room (predicated, no branch), then
-// close the group.
+// close the group.  A block landing in slot 0 is also copied to the mirror
+// slot after slot 3, so that a step's reads run past the end of slot 3 without
+// wrapping.
 __device__ __forceinline__ void ring_issue(Ring& r, uint32_t p) {
   const uint32_t want = min((p >> 3) + kRingBlocks, r.lim);
   const uint32_t dst = r.rb + (r.fb & (kRingBlocks - 1)) * 16u;
   const uint8_t* src = r.gbase + uint64_t(r.fb) * 16u;
   asm volatile(
       "{\n\t"
-      ".reg .pred p;\n\t"
+      ".reg .pred p, m;\n\t"
+      ".reg .u32 t;\n\t"
       "setp.lt.u32 p, %0, %1;\n\t"
+      "and.b32 t, %0, 3;\n\t"
+      "setp.eq.and.u32 m, t, 0, p;\n\t"
       "@p cp.async.cg.shared.global [%2], [%3], 16;\n\t"
+      "@m cp.async.cg.shared.global [%4], [%3], 16;\n\t"
       "@p add.u32 %0, %0, 1;\n\t"
       "cp.async.commit_group;\n\t"
       "}\n"
       : "+r"(r.fb)
-      : "r"(want), "r"(dst), "l"(src)
+      : "r"(want), "r"(dst), "l"(src), "r"(r.rb + kRingBytes)
       : "memory");
 }
 
@@ -219,25 +225,30 @@ __device__ __forceinline__ void fill_table(uint32_t* tbl, CumBuf cb, int tid) {
 
 // One rANS decode step: returns the packed table entry of the decoded symbol.
 // The refill is predicated, not branched: x = (x << 16) | w, advance the ring
-// address ra (wrapping inside the thread's 64 bytes) and load the next word.
+// address ra and load the next word.  Within a step ra never wraps: it starts
+// the step inside the 64-byte ring and a step reads at most 16 bytes, which
+// may run into the mirror of slot 0.
 __device__ __forceinline__ uint32_t rans_step(uint32_t& x, uint32_t& ra, uint32_t& w,
-                                              const uint32_t* __restrict__ tbl, uint32_t rb) {
+                                              const uint32_t* __restrict__ tbl) {
   const uint32_t e = tbl[x & (kM - 1)];
   x = ((e >> 12) & (kM - 1)) * (x >> kProbBits) + (e & (kM - 1));
   asm volatile(
       "{\n\t"
       ".reg .pred p;\n\t"
-      ".reg .u32 t;\n\t"
-      "setp.lt.u32 p, %0, %4;\n\t"
+      "setp.lt.u32 p, %0, %3;\n\t"
       "@p prmt.b32 %0, %2, %0, 0x5410;\n\t"
-      "@p add.u32 t, %1, 2;\n\t"
-      "@p and.b32 t, t, 63;\n\t"
-      "@p or.b32 %1, t, %3;\n\t"
+      "@p add.u32 %1, %1, 2;\n\t"
       "@p ld.shared.u16 %2, [%1];\n\t"
       "}\n"
       : "+r"(x), "+r"(ra), "+r"(w)
-      : "r"(rb), "n"(kRansL));
+      : "n"(kRansL));
   return e;
+}
+
+// Start of a step: bring the read address back into the 64-byte ring (the word
+// under it is the same in slot 0 and in its mirror).
+__device__ __forceinline__ uint32_t ring_rebase(uint32_t ra, uint32_t rb) {
+  return rb + ((ra - rb) & (kRingBytes - 1));
 }
 
 // (float)(u - 127) for the symbol u in the entry's top byte: the bits
@@ -284,19 +295,20 @@ __device__ __forceinline__ void decode_delta_head(uint32_t& x, Pos& ps, Ring& r,
       const int dd = d0 + 8 * half;
       ring_issue(r, ps.p);
       ring_wait_two_steps();
+      ps.ra = ring_rebase(ps.ra, r.rb);
       const uint32_t ra0 = ps.ra;
       const float4 a0 = *reinterpret_cast<const float4*>(arow + dd);
       const float4 a1 = *reinterpret_cast<const float4*>(arow + dd + 4);
       const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
       for (int k = 0; k < 8; k += 2) {
-        const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+        const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl);
         const float v0 = __fadd_rn(a[k], __fmul_rn(sym_value(e0), step));
-        const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+        const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl);
         const float v1 = __fadd_rn(a[k + 1], __fmul_rn(sym_value(e1), step));
         hv[4 * half + (k >> 1)] = pack_half2(v0, v1);
       }
-      ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
+      ps.p += (ps.ra - ra0) >> 1;
     }
     store16h(orow + d0, hv, al32);
   }
@@ -317,6 +329,7 @@ __device__ __forceinline__ void decode_anchor_head(uint32_t& x, Pos& ps, Ring& r
       const int dd = d0 + 8 * half;
       ring_issue(r, ps.p);
       ring_wait_two_steps();
+      ps.ra = ring_rebase(ps.ra, r.rb);
       const uint32_t ra0 = ps.ra;
       const float4 z0 = *reinterpret_cast<const float4*>(zp + dd);
       const float4 z1 = *reinterpret_cast<const float4*>(zp + dd + 4);
@@ -327,10 +340,10 @@ __device__ __forceinline__ void decode_anchor_head(uint32_t& x, Pos& ps, Ring& r
       float v[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const uint32_t e = rans_step(x, ps.ra, ps.w, tbl, r.rb);
+        const uint32_t e = rans_step(x, ps.ra, ps.w, tbl);
         v[k] = __fadd_rn(z[k], __fmul_rn(sym_value(e), s[k]));
       }
-      ps.p += ((ps.ra - ra0) & (kRingBytes - 1)) >> 1;
+      ps.p += (ps.ra - ra0) >> 1;
       *reinterpret_cast<float4*>(arow + dd) = make_float4(v[0], v[1], v[2], v[3]);
       *reinterpret_cast<float4*>(arow + dd + 4) = make_float4(v[4], v[5], v[6], v[7]);
 #pragma unroll
@@ -456,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   const uint32_t* offs = reinterpret_cast<const uint32_t*>(base + sec.offsets);
   Ring ring;
   ring.gbase = base;
-  const uint32_t rings = (uint32_t(__cvta_generic_to_shared(smem + sm.ring)) + 63u) & ~63u;
-  ring.rb = rings + uint32_t(tid) * kRingBytes;
+  const uint32_t rings = uint32_t(__cvta_generic_to_shared(smem + sm.ring));
+  ring.rb = rings + uint32_t(tid) * kRingStride;
   ring.lim = uint32_t(s_total / 16);
   ring.fb = 0;
   Pos ps{0u, ring.rb, 0u};
