@@ -113,6 +113,23 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+def reduce_max(values, world, dist, device):
+    """Max over ranks of each entry (the job's time is its slowest rank's);
+    a no-op for one rank.  `device` is where the collective runs (the rank's
+    GPU under NCCL, the CPU under gloo)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_gbps(bytes_per_rank, world, ms):
+    """Whole-job throughput: the bytes of all ranks over the max-over-ranks time."""
+    return bytes_per_rank * world / ms / 1e6
+
+
 def _oracle_sample(threads: int):
     """The CPU sample: one chunk of the workload cut into 16 independent 2-head
     slices ([32, 2, 1536, 2, 128] each, 50 MB of fp16), round-tripped through the
@@ -238,12 +255,7 @@ def run_ours(args):
     t_enc = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
     t_dec = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
     t_step = sum(t_enc) + sum(t_dec)
-    if world > 1:
-        tt = torch.tensor([t_step, sum(t_enc), sum(t_dec)], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step, te_sum, td_sum = tt.tolist()
-    else:
-        te_sum, td_sum = sum(t_enc), sum(t_dec)
+    t_step, te_sum, td_sum = reduce_max([t_step, sum(t_enc), sum(t_dec)], world, dist, dev)
     ms_step = t_step / args.steps
     ms_enc = te_sum / args.steps
     ms_dec = td_sum / args.steps
@@ -267,7 +279,7 @@ def run_ours(args):
     if rank == 0:
         line = {
             "metric": METRIC,
-            "value": round(fp16_bytes * world / ms_step / 1e6, 2),
+            "value": round(job_gbps(fp16_bytes, world, ms_step), 2),
             "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_step, 4),
@@ -345,15 +357,11 @@ def _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, 
     torch.cuda.synchronize(dev)
     if int(host_status[0]) != 0 or int(host_status[1]) != 0:
         raise RuntimeError(f"e2e status {host_status.tolist()}")
-    ms = t0.elapsed_time(t1) / steps
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = reduce_max([t0.elapsed_time(t1) / steps], world, dist, dev)[0]
     comp = sum(sizes)
     h2d = fp16_bytes + comp
     d2h = comp + 8
-    return {"value": round(fp16_bytes * world / ms / 1e6, 3), "unit": "GB/s",
+    return {"value": round(job_gbps(fp16_bytes, world, ms), 3), "unit": "GB/s",
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
