@@ -161,6 +161,13 @@ def _oracle_sample(threads: int):
             sizes = list(ex.map(run_one, slices))
         return time.perf_counter() - t0, sizes
 
+    def one_core():
+        """One slice on the calling thread: the oracle's single-core rate."""
+        t0 = time.perf_counter()
+        run_one(slices[0])
+        return time.perf_counter() - t0, slices[0].nbytes
+
+    step.one_core = one_core
     return step, nbytes, desc
 
 
@@ -369,8 +376,11 @@ def _cpu_baseline():
     threads = max(1, min(16, os.cpu_count() or 1))
     step, nbytes, desc = _oracle_sample(threads)
     dt, _ = step()
+    dt1, nb1 = step.one_core()
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle", "sample": desc}
+            "kind": "oracle", "sample": desc,
+            "single_core": {"value": round(nb1 / dt1 / 1e9, 4), "unit": "GB/s",
+                            "sample": "the first of the 16 slices on one thread"}}
 
 
 def main():
