@@ -233,6 +233,25 @@ cg_status cg_decode_into(const cg_shape* shape, const uint8_t* in_dev, uint64_t 
                          uint16_t* kv_dev, int64_t total_tokens, int32_t* status_dev,
                          cudaStream_t stream);
 
+/* As cg_decode_into, but into a paged KV pool, the layout of serving engines
+ * that hand out the cache in fixed-size token pages through a block table.
+ * pool_dev holds num_pages pages of page_tokens tokens for every (layer, K/V):
+ * [L][2][num_pages][page_tokens][H][D] (16-byte aligned).  Logical token t
+ * (0 <= t < total_tokens, the sequence's capacity) lives in row
+ * t % page_tokens of page block_table_dev[t / page_tokens]; block_table_dev
+ * (int32, device, read only) has ceil(total_tokens / page_tokens) entries.
+ * Each chunk lands at the token_start stored in its header, which must satisfy
+ * token_start + n <= total_tokens (else CG_ERR_MISMATCH).  A block-table entry
+ * outside [0, num_pages) sets CG_ERR_MISMATCH and nothing is written for the
+ * tokens of that page.  Grounding: [Practice] 2.3 (the fill thread that
+ * injects decoded KV into the model's cache); the page layout is the
+ * integration this call serves, the pages do not fix it. */
+cg_status cg_decode_into_paged(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
+                               int32_t num_chunks, int32_t chunk_tokens, cg_level level,
+                               uint16_t* pool_dev, int32_t num_pages, int32_t page_tokens,
+                               const int32_t* block_table_dev, int64_t total_tokens,
+                               int32_t* status_dev, cudaStream_t stream);
+
 /* cg_encode without caller-provided scratch.  The pages have no counterpart
  * to this call; it exists for callers that cannot allocate device memory --
  * an inference server that has reserved the whole GPU for its own pool, a

@@ -214,8 +214,13 @@ cg_status cg_encode(const cg_shape* shape, const uint16_t* kv_dev, int64_t total
 static cg_status decode_common(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
                                int32_t num_chunks, int32_t chunk_tokens, cg_level level,
                                uint16_t* out_dev, uint64_t out_elems, int into,
-                               int64_t total_tokens, int32_t* status_dev, cudaStream_t stream) {
+                               int64_t total_tokens, int32_t* status_dev, cudaStream_t stream,
+                               const int32_t* block_table = nullptr, int32_t num_pages = 0,
+                               int32_t page_tokens = 0) {
   cg::DecParams p{};
+  p.block_table = block_table;
+  p.num_pages = num_pages;
+  p.page_tokens = page_tokens;
   p.in = in_dev;
   p.in_stride = in_stride;
   p.num_chunks = num_chunks;
@@ -258,6 +263,23 @@ cg_status cg_decode_into(const cg_shape* shape, const uint8_t* in_dev, uint64_t 
                          shape->num_kv_heads * shape->head_dim;
   return decode_common(shape, in_dev, in_stride, num_chunks, chunk_tokens, level, kv_dev, elems,
                        1, total_tokens, status_dev, stream);
+}
+
+cg_status cg_decode_into_paged(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
+                               int32_t num_chunks, int32_t chunk_tokens, cg_level level,
+                               uint16_t* pool_dev, int32_t num_pages, int32_t page_tokens,
+                               const int32_t* block_table_dev, int64_t total_tokens,
+                               int32_t* status_dev, cudaStream_t stream) {
+  cg_status st = check_decode_args(shape, in_dev, in_stride, num_chunks, chunk_tokens, level,
+                                   pool_dev, status_dev);
+  if (st != CG_OK) return st;
+  if (total_tokens < 1 || num_pages < 1 || page_tokens < 1 || block_table_dev == nullptr)
+    return CG_ERR_INVALID_ARG;
+  const uint64_t elems = uint64_t(shape->num_layers) * 2 * uint64_t(num_pages) *
+                         uint64_t(page_tokens) * shape->num_kv_heads * shape->head_dim;
+  return decode_common(shape, in_dev, in_stride, num_chunks, chunk_tokens, level, pool_dev,
+                       elems, 2, total_tokens, status_dev, stream, block_table_dev, num_pages,
+                       page_tokens);
 }
 
 }  // extern "C"

@@ -137,8 +137,12 @@ struct DecParams {
   int level;
   uint16_t* out;
   uint64_t out_elems;      // size of out in elements (bounds every store)
-  int into;                // 0: chunk slots [L][2][n][H][D]; 1: full KV [L][2][T][H][D]
-  int64_t total_tokens;    // T of the full KV (into mode)
+  int into;                // 0: chunk slots [L][2][n][H][D]; 1: full KV [L][2][T][H][D];
+                           // 2: paged pool [L][2][num_pages][page_tokens][H][D]
+  int64_t total_tokens;    // T of the full KV (modes 1 and 2)
+  const int32_t* block_table;  // mode 2: physical page of logical page t / page_tokens
+  int num_pages;           // mode 2
+  int page_tokens;         // mode 2
   int units_per_slab;      // CTAs per (chunk, l, kv)
   int32_t* status;
 };

@@ -467,6 +467,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   }
   bool active = token < n;
   const uint32_t* offs = reinterpret_cast<const uint32_t*>(base + sec.offsets);
+  // Destination row of this thread's token.
+  uint16_t* orow = p.out;
+  if (p.into == 1) {
+    orow = p.out + ((uint64_t(slab) * p.total_tokens + uint64_t(s_tstart) + token) * H) * D;
+  } else if (p.into == 2) {
+    // paged pool: logical token t is row t mod P of page block_table[t / P]
+    const int64_t t = s_tstart + token;
+    const int32_t page = active ? __ldg(p.block_table + t / p.page_tokens) : 0;
+    if (page < 0 || page >= p.num_pages) {
+      set_status(p.status, CG_ERR_MISMATCH);
+      active = false;
+    } else {
+      orow = p.out + (((uint64_t(slab) * p.num_pages + uint64_t(page)) * p.page_tokens +
+                       uint64_t(t % p.page_tokens)) * H) * D;
+    }
+  } else {
+    orow = p.out + uint64_t(chunk) * (uint64_t(L) * 2 * p.C * H * D) +
+           ((uint64_t(slab) * n + token) * H) * D;
+  }
   Ring ring;
   ring.gbase = base;
   const uint32_t rings = uint32_t(__cvta_generic_to_shared(smem + sm.ring));
@@ -499,12 +518,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
       }
     }
   }
-  uint16_t* orow;
-  if (p.into)
-    orow = p.out + ((uint64_t(slab) * p.total_tokens + uint64_t(s_tstart) + token) * H) * D;
-  else
-    orow = p.out + uint64_t(chunk) * (uint64_t(L) * 2 * p.C * H * D) +
-           ((uint64_t(slab) * n + token) * H) * D;
   const float* zp_sec = reinterpret_cast<const float*>(base + sec.zp) + size_t(slab) * H * D;
   const float* sc_sec = reinterpret_cast<const float*>(base + sec.scale) + size_t(slab) * H * D;
   float* zs = reinterpret_cast<float*>(smem + sm.zs);  // [2][{zp, scale}][D]

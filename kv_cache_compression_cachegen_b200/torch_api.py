@@ -13,7 +13,8 @@ from dataclasses import dataclass
 import torch
 
 from . import (CG_OK, CacheGenError, Shape, cg_build_tables, cg_decode, cg_decode_into,
-               cg_encode, cg_encode_workspace_bytes, cg_encoded_bound, cg_tables_bytes, check)
+               cg_decode_into_paged, cg_encode, cg_encode_workspace_bytes, cg_encoded_bound,
+               cg_tables_bytes, check)
 
 
 def _shape_of(kv: torch.Tensor) -> tuple[Shape, int]:
@@ -120,6 +121,22 @@ def decode_into(data: torch.Tensor, stride: int, shape: Shape, chunk_tokens: int
         status = new_status(data.device)
     check(cg_decode_into(shape, data, stride, num_chunks, chunk_tokens, level, kv, T, status,
                          stream), "cg_decode_into")
+    return status
+
+
+def decode_into_paged(data: torch.Tensor, stride: int, shape: Shape, chunk_tokens: int,
+                      level: int, num_chunks: int, pool: torch.Tensor, page_tokens: int,
+                      block_table: torch.Tensor, total_tokens: int,
+                      status: torch.Tensor | None = None, stream=None):
+    """Decode into a paged pool [L][2][num_pages][page_tokens][H][D] through an
+    int32 block table (logical page -> physical page)."""
+    L, H, D = shape.num_layers, shape.num_kv_heads, shape.head_dim
+    num_pages = pool.numel() // (L * 2 * page_tokens * H * D)
+    if status is None:
+        status = new_status(data.device)
+    check(cg_decode_into_paged(shape, data, stride, num_chunks, chunk_tokens, level, pool,
+                               num_pages, page_tokens, block_table, total_tokens, status,
+                               stream), "cg_decode_into_paged")
     return status
 
 

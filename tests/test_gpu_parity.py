@@ -173,3 +173,38 @@ def test_destination_only_16_byte_aligned():
     for k in range(nch):
         n = min(C, T - k * C)
         assert torch.equal(kv2[:, :, k * C:k * C + n], gu.chunk_slot(ref, shape, C, k, n))
+
+
+def test_decode_into_paged_pool():
+    # A shuffled block table: decoding into the paged pool must put every token's
+    # row exactly where the flat decode_into puts it, page by page.
+    L, H, D, T, C, P = 3, 2, 64, 250, 96, 16
+    kv = gu.gen(L, H, D, T, seed=13)
+    shape = Shape(L, H, D)
+    nch = -(-T // C)
+    enc = ta.encode(kv, C, 2)
+    flat = torch.full_like(kv, 0x7E00)
+    st = ta.decode_into(enc.data, enc.stride, shape, C, 2, nch, flat)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == 0
+    npages_logical = -(-T // P)
+    num_pages = npages_logical + 5
+    g = torch.Generator().manual_seed(3)
+    table = torch.randperm(num_pages, generator=g)[:npages_logical].to(torch.int32).cuda()
+    pool = torch.full((L, 2, num_pages, P, H, D), 0x7E00, dtype=torch.int16, device="cuda")
+    st = ta.decode_into_paged(enc.data, enc.stride, shape, C, 2, nch, pool, P, table, T)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == 0
+    tab = table.cpu().tolist()
+    for lp in range(npages_logical):
+        a, b = lp * P, min(T, (lp + 1) * P)
+        assert torch.equal(pool[:, :, tab[lp], :b - a], flat[:, :, a:b]), lp
+    # pages no logical page maps to stay untouched
+    unused = sorted(set(range(num_pages)) - set(tab))
+    assert bool((pool[:, :, unused] == 0x7E00).all())
+    # a block-table entry outside the pool is a mismatch
+    bad = table.clone()
+    bad[2] = num_pages
+    st = ta.decode_into_paged(enc.data, enc.stride, shape, C, 2, nch, pool, P, bad, T)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == CG_ERR_MISMATCH

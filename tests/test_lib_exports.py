@@ -56,4 +56,9 @@ def test_argument_errors_are_synchronous(native_built):
     assert cg.cg_decode(shp, None, 64, 1, 256, 1, None, 0, None, stream=0) == cg.CG_ERR_INVALID_ARG
     assert cg.cg_decode_into(shp, 16, 64, 1, 256, 5, 16, 256, 16, stream=0) == cg.CG_ERR_INVALID_ARG
     assert cg.cg_build_tables(shp, 16, 256, 0, 2, 256, 1, 16, 16, stream=0) == cg.CG_ERR_INVALID_ARG
+    # paged decode: no block table, or an empty pool
+    assert cg.cg_decode_into_paged(shp, 16, 64, 1, 256, 1, 16, 4, 16, None, 64, 16,
+                                   stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_decode_into_paged(shp, 16, 64, 1, 256, 1, 16, 0, 16, 16, 64, 16,
+                                   stream=0) == cg.CG_ERR_INVALID_ARG
     assert cg.cg_status_string(cg.CG_ERR_CORRUPT) == "corrupt container"
