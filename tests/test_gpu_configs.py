@@ -131,3 +131,35 @@ def test_chunk_size_and_distribution_sweep(dist):
             dref = _compare_sampled(kv, enc, C, level, [last])
             n = w.T - last * C
             assert np.array_equal(gu.host(out[:, :, last * C:last * C + n]), dref[last])
+
+
+def test_bandwidth_adaptive_stream_decode():
+    """Three versions per chunk, a bandwidth trace picks each chunk's version, the
+    chunks stream in (copy of the next overlapping the decode of the current),
+    and every chunk equals the decode of the version that was sent."""
+    from kv_cache_compression_cachegen_b200 import streaming
+    L, H, D, C = 4, 2, 64, 256
+    T = 7 * C + 100
+    kv = gu.gen(L, H, D, T, seed=21)
+    shape = Shape(L, H, D)
+    store = streaming.encode_all_levels(kv, C)
+    trace = [8.0, 3.0, 0.5, 6.0, 1.0, 0.2, 4.0, 9.0]
+    levels = streaming.plan_levels(trace)
+    assert len(levels) == store.num_chunks
+    out = torch.full_like(kv, 0x7E00)
+    status = streaming.stream_decode(store, levels, out)
+    torch.cuda.synchronize()
+    assert ta.status_of(status) == 0
+    for k in range(store.num_chunks):
+        buf = store.containers[(levels[k], k)].cuda()
+        slot, st = ta.decode(buf, buf.numel(), shape, C, levels[k], 1)
+        torch.cuda.synchronize()
+        assert ta.status_of(st) == 0
+        n = min(C, T - k * C)
+        assert torch.equal(out[:, :, k * C:k * C + n], gu.chunk_slot(slot, shape, C, 0, n))
+    # the balanced versions also match the oracle
+    kv_h = gu.host(kv)
+    k = levels.index(1)
+    ref = gu.oracle_containers(kv_h, C, 1, [k])
+    got = store.containers[(1, k)].numpy()[:ref[k].size]
+    assert np.array_equal(got, ref[k])
