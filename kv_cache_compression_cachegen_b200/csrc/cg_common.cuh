@@ -136,7 +136,7 @@ struct DecParams {
   int C, L, H, D;
   int level;
   uint16_t* out;
-  uint64_t out_elems;      // size of out in elements (bounds every store)
+  uint64_t out_elems;      // size of out in elements (checked against the shape by the C ABI)
   int into;                // 0: chunk slots [L][2][n][H][D]; 1: full KV [L][2][T][H][D];
                            // 2: paged pool [L][2][num_pages][page_tokens][H][D]
   int64_t total_tokens;    // T of the full KV (modes 1 and 2)
