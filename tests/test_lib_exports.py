@@ -56,6 +56,13 @@ def test_argument_errors_are_synchronous(native_built):
     assert cg.cg_decode(shp, None, 64, 1, 256, 1, None, 0, None, stream=0) == cg.CG_ERR_INVALID_ARG
     assert cg.cg_decode_into(shp, 16, 64, 1, 256, 5, 16, 256, 16, stream=0) == cg.CG_ERR_INVALID_ARG
     assert cg.cg_build_tables(shp, 16, 256, 0, 2, 256, 1, 16, 16, stream=0) == cg.CG_ERR_INVALID_ARG
+    # empty calls: no chunk, no token
+    assert cg.cg_encode(shp, 16, 256, 0, 0, 256, 1, None, 16, 4096, 16, 16, 256, 1 << 20,
+                        stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_encode(shp, 16, 0, 0, 1, 256, 1, None, 16, 4096, 16, 16, 256, 1 << 20,
+                        stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_decode(shp, 16, 4096, 0, 256, 1, 16, 1 << 20, 16, stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_decode_into(shp, 16, 4096, 1, 256, 1, 16, 0, 16, stream=0) == cg.CG_ERR_INVALID_ARG
     # paged decode: no block table, or an empty pool
     assert cg.cg_decode_into_paged(shp, 16, 64, 1, 256, 1, 16, 4, 16, None, 64, 16,
                                    stream=0) == cg.CG_ERR_INVALID_ARG
