@@ -76,6 +76,15 @@ def lib() -> ctypes.CDLL:
             "orc_decode_chunk": (_c.c_int, [_u8p, _c.c_uint64, _c.c_int, _c.c_int, _c.c_int,
                                             _c.c_int, _c.c_int, _u16p, _c.c_uint64,
                                             _c.POINTER(_c.c_int64), _c.POINTER(_c.c_int64)]),
+            "orc_quantize_chunk_v": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _u16p, _c.c_int64,
+                                                _c.c_int64, _c.c_int, _c.c_int, _c.c_int, _u8p,
+                                                _f32p, _f32p]),
+            "orc_encode_chunk_v": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _u16p, _c.c_int64,
+                                              _c.c_int64, _c.c_int, _c.c_int, _c.c_int, _u8p,
+                                              _c.c_uint64, _c.POINTER(_c.c_uint64)]),
+            "orc_decode_chunk_v": (_c.c_int, [_u8p, _c.c_uint64, _c.c_int, _c.c_int, _c.c_int,
+                                              _c.c_int, _c.c_int, _c.c_int, _u16p, _c.c_uint64,
+                                              _c.POINTER(_c.c_int64), _c.POINTER(_c.c_int64)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -180,15 +189,17 @@ def encoded_bound(L: int, H: int, D: int, C: int) -> int:
     return int(lib().orc_encoded_bound(L, H, D, C))
 
 
-def quantize_chunk(kv: np.ndarray, token_start: int, C: int, level: int):
-    """kv: uint16 [L, 2, T, H, D].  Returns (status, sym [L,2,n,H,D], zp, scale)."""
+def quantize_chunk(kv: np.ndarray, token_start: int, C: int, level: int,
+                   adjacent: bool = False):
+    """kv: uint16 [L, 2, T, H, D].  Returns (status, sym [L,2,n,H,D], zp, scale).
+    adjacent=True: format 2, deltas to the previous token's reconstruction."""
     L, _, T, H, D = kv.shape
     n = min(C, T - token_start)
     sym = np.zeros((L, 2, n, H, D), dtype=np.uint8)
     zp = np.zeros((L, 2, H, D), dtype=np.float32)
     sc = np.zeros((L, 2, H, D), dtype=np.float32)
-    rc = lib().orc_quantize_chunk(L, H, D, np.ascontiguousarray(kv, dtype=np.uint16), T,
-                                  token_start, C, level, sym, zp, sc)
+    rc = lib().orc_quantize_chunk_v(L, H, D, np.ascontiguousarray(kv, dtype=np.uint16), T,
+                                    token_start, C, level, int(adjacent), sym, zp, sc)
     return rc, sym, zp, sc
 
 
@@ -199,23 +210,28 @@ def tables_of(sym: np.ndarray) -> np.ndarray:
     return freq
 
 
-def encode_chunk(kv: np.ndarray, token_start: int, C: int, level: int):
-    """Returns (status, container bytes as uint8 array)."""
+def encode_chunk(kv: np.ndarray, token_start: int, C: int, level: int,
+                 adjacent: bool = False):
+    """Returns (status, container bytes as uint8 array); adjacent=True writes
+    format 2 (header version 2)."""
     L, _, T, H, D = kv.shape
     cap = encoded_bound(L, H, D, C)
     out = np.zeros(cap, dtype=np.uint8)
     size = _c.c_uint64(0)
-    rc = lib().orc_encode_chunk(L, H, D, np.ascontiguousarray(kv, dtype=np.uint16), T,
-                                token_start, C, level, out, cap, _c.byref(size))
+    rc = lib().orc_encode_chunk_v(L, H, D, np.ascontiguousarray(kv, dtype=np.uint16), T,
+                                  token_start, C, level, int(adjacent), out, cap,
+                                  _c.byref(size))
     return rc, out[: size.value].copy()
 
 
-def decode_chunk(container, L: int, H: int, D: int, C: int, level: int):
-    """Returns (status, values uint16 [L,2,n,H,D], n, token_start)."""
+def decode_chunk(container, L: int, H: int, D: int, C: int, level: int,
+                 adjacent: bool = False):
+    """Returns (status, values uint16 [L,2,n,H,D], n, token_start).  The
+    container's format must be the one asked for (else MISMATCH)."""
     buf = np.ascontiguousarray(container, dtype=np.uint8)
     out = np.zeros(L * 2 * C * H * D, dtype=np.uint16)
     n, start = _c.c_int64(0), _c.c_int64(0)
-    rc = lib().orc_decode_chunk(buf, buf.size, L, H, D, C, level, out, out.size, _c.byref(n),
-                                _c.byref(start))
+    rc = lib().orc_decode_chunk_v(buf, buf.size, L, H, D, C, level, int(adjacent), out,
+                                  out.size, _c.byref(n), _c.byref(start))
     vals = out[: L * 2 * n.value * H * D].reshape(L, 2, n.value, H, D) if rc == OK else out[:0]
     return rc, vals, n.value, start.value

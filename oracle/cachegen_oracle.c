@@ -21,6 +21,12 @@
  * fixes where the pages are silent.  Every step below is written in the
  * order the method applies it, with no blocking or fusion.
  *
+ * Two container formats: format 1 codes every token of a group as a delta to
+ * the group's reconstructed anchor; format 2 reads [Practice] 1 literally
+ * ("the difference between adjacent tokens") and codes token t as a delta to
+ * the reconstruction of token t - 1, restarting at every anchor.  The formats
+ * differ only in that reference and in the header's version field.
+ *
  * Compiled with -O2 -ffp-contract=off and without -ffast-math, so every
  * float expression is one IEEE round-to-nearest operation per operator.
  *
@@ -351,9 +357,15 @@ static size_t kv_index(int64_t T, int H, int D, int l, int kv, int64_t t, int h,
   return ((((size_t)l * 2 + kv) * (size_t)T + (size_t)t) * H + h) * (size_t)D + d;
 }
 
-int orc_quantize_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
-                       int C, int level, uint8_t* sym, float* zp, float* scale) {
+/* adjacent == 0 (format 1): every token of a group is a delta to the group's
+ * reconstructed anchor.  adjacent == 1 (format 2, [Practice] 1 read
+ * literally: "the difference between adjacent tokens"): every token is a
+ * delta to the reconstruction of the token just before it, x^_t =
+ * x^_(t-1) + q_t * step, and the chain restarts at each group's anchor. */
+int orc_quantize_chunk_v(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
+                         int C, int level, int adjacent, uint8_t* sym, float* zp, float* scale) {
   if (L < 1 || H < 1 || D < 1 || C < 1 || level < 0 || level > 2) return ORC_INVALID;
+  if (adjacent != 0 && adjacent != 1) return ORC_INVALID;
   if (token_start < 0 || token_start >= T) return ORC_INVALID;
   int64_t n = T - token_start;
   if (n > C) n = C;
@@ -383,10 +395,12 @@ int orc_quantize_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64
             float ahat = orc_anchor_value(c, zp[ch], scale[ch]);
             int64_t t0 = g * ORC_GROUP;
             sym[kv_index(n, H, D, l, kvi, t0, h, d)] = (uint8_t)(c + 127);
+            float ref = ahat; /* what the next delta is taken against */
             for (int64_t t = t0 + 1; t < t0 + ORC_GROUP && t < n; t++) {
               float x = orc_f16_to_f32(kv[kv_index(T, H, D, l, kvi, token_start + t, h, d)]);
-              int q = orc_delta_code(x, ahat, step);
+              int q = orc_delta_code(x, ref, step);
               sym[kv_index(n, H, D, l, kvi, t, h, d)] = (uint8_t)(q + 127);
+              if (adjacent) ref = orc_delta_value(q, ref, step);
             }
           }
         }
@@ -395,6 +409,11 @@ int orc_quantize_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64
   }
   free(anchors);
   return ORC_OK;
+}
+
+int orc_quantize_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
+                       int C, int level, uint8_t* sym, float* zp, float* scale) {
+  return orc_quantize_chunk_v(L, H, D, kv, T, token_start, C, level, 0, sym, zp, scale);
 }
 
 /* Frequency tables [L][2][H][256] of a quantised chunk. */
@@ -414,9 +433,11 @@ void orc_tables_of(int L, int H, int D, int64_t n, const uint8_t* sym, uint16_t*
 /* Encode one chunk into a container ([Practice] 2.1: each chunk is encoded on
  * its own; [Practice] 1: quantise, then entropy-code). */
 
-int orc_encode_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
-                     int C, int level, uint8_t* out, uint64_t cap, uint64_t* out_size) {
+int orc_encode_chunk_v(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
+                       int C, int level, int adjacent, uint8_t* out, uint64_t cap,
+                       uint64_t* out_size) {
   if (L < 1 || H < 1 || D < 1 || C < 1 || level < 0 || level > 2) return ORC_INVALID;
+  if (adjacent != 0 && adjacent != 1) return ORC_INVALID;
   if (token_start < 0 || token_start >= T) return ORC_INVALID;
   int64_t n = T - token_start;
   if (n > C) n = C;
@@ -434,7 +455,7 @@ int orc_encode_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t
     rc = ORC_INVALID;
     goto done;
   }
-  rc = orc_quantize_chunk(L, H, D, kv, T, token_start, C, level, sym, zp, scale);
+  rc = orc_quantize_chunk_v(L, H, D, kv, T, token_start, C, level, adjacent, sym, zp, scale);
   if (rc != ORC_OK) goto done;
   orc_tables_of(L, H, D, n, sym, freq);
 
@@ -484,7 +505,7 @@ int orc_encode_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t
 
   memset(out, 0, ORC_HEADER);
   put32(out + 0, ORC_MAGIC);
-  put16(out + 4, 1);
+  put16(out + 4, (uint16_t)(1 + adjacent)); /* format 1: anchor deltas; 2: adjacent */
   out[6] = (uint8_t)level;
   out[7] = ORC_GROUP;
   put32(out + 8, (uint32_t)L);
@@ -509,15 +530,25 @@ done:
   return rc;
 }
 
+int orc_encode_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
+                     int C, int level, uint8_t* out, uint64_t cap, uint64_t* out_size) {
+  return orc_encode_chunk_v(L, H, D, kv, T, token_start, C, level, 0, out, cap, out_size);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Decode one container ([Practice] 2.3: decode, then fill the model's KV).
  * Values go to out[L][2][n][H][D] (out_elems must hold them). */
 
-int orc_decode_chunk(const uint8_t* in, uint64_t in_bytes, int L, int H, int D, int C, int level,
-                     uint16_t* out, uint64_t out_elems, int64_t* n_out, int64_t* start_out) {
+int orc_decode_chunk_v(const uint8_t* in, uint64_t in_bytes, int L, int H, int D, int C,
+                       int level, int adjacent, uint16_t* out, uint64_t out_elems,
+                       int64_t* n_out, int64_t* start_out) {
+  if (adjacent != 0 && adjacent != 1) return ORC_INVALID;
   if (in_bytes < ORC_HEADER) return ORC_CORRUPT;
-  if (get32(in) != ORC_MAGIC || get16(in + 4) != 1 || in[7] != ORC_GROUP || get32(in + 28) != 12)
+  int version = get16(in + 4);
+  if (get32(in) != ORC_MAGIC || (version != 1 && version != 2) || in[7] != ORC_GROUP ||
+      get32(in + 28) != 12)
     return ORC_CORRUPT;
+  if (version != 1 + adjacent) return ORC_MISMATCH; /* the other delta format */
   if (in[6] != level || get32(in + 8) != (uint32_t)L || get32(in + 12) != (uint32_t)H ||
       get32(in + 16) != (uint32_t)D || get32(in + 20) != (uint32_t)C)
     return ORC_MISMATCH;
@@ -590,10 +621,12 @@ int orc_decode_chunk(const uint8_t* in, uint64_t in_bytes, int L, int H, int D, 
             int c = (int)sym[((size_t)t0 * H + h) * D + d] - 127;
             float ahat = orc_anchor_value(c, zp, scale);
             out[kv_index(n, H, D, l, kvi, t0, h, d)] = orc_f32_to_f16(ahat);
+            float ref = ahat;
             for (int64_t t = t0 + 1; t < t0 + ORC_GROUP && t < n; t++) {
               int q = (int)sym[((size_t)t * H + h) * D + d] - 127;
-              out[kv_index(n, H, D, l, kvi, t, h, d)] =
-                  orc_f32_to_f16(orc_delta_value(q, ahat, step));
+              float v = orc_delta_value(q, ref, step);
+              out[kv_index(n, H, D, l, kvi, t, h, d)] = orc_f32_to_f16(v);
+              if (adjacent) ref = v; /* format 2: the next delta builds on this token */
             }
           }
         }
@@ -607,6 +640,11 @@ done:
   free(slots);
   free(words);
   return rc;
+}
+
+int orc_decode_chunk(const uint8_t* in, uint64_t in_bytes, int L, int H, int D, int C, int level,
+                     uint16_t* out, uint64_t out_elems, int64_t* n_out, int64_t* start_out) {
+  return orc_decode_chunk_v(in, in_bytes, L, H, D, C, level, 0, out, out_elems, n_out, start_out);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -44,4 +44,16 @@ int orc_encode_chunk(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t
 int orc_decode_chunk(const uint8_t* in, uint64_t in_bytes, int L, int H, int D, int C, int level,
                      uint16_t* out, uint64_t out_elems, int64_t* n_out, int64_t* start_out);
 
+/* Format variants: adjacent = 0 is format 1 (deltas to the group's anchor);
+ * adjacent = 1 is format 2 (deltas to the previous token's reconstruction,
+ * header version 2).  The functions above are the adjacent = 0 forms. */
+int orc_quantize_chunk_v(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
+                         int C, int level, int adjacent, uint8_t* sym, float* zp, float* scale);
+int orc_encode_chunk_v(int L, int H, int D, const uint16_t* kv, int64_t T, int64_t token_start,
+                       int C, int level, int adjacent, uint8_t* out, uint64_t cap,
+                       uint64_t* out_size);
+int orc_decode_chunk_v(const uint8_t* in, uint64_t in_bytes, int L, int H, int D, int C,
+                       int level, int adjacent, uint16_t* out, uint64_t out_elems,
+                       int64_t* n_out, int64_t* start_out);
+
 #endif
