@@ -113,7 +113,8 @@
 extern "C" {
 #endif
 
-#define CG_FORMAT_VERSION 1
+#define CG_FORMAT_VERSION 1          /* deltas to the group's reconstructed anchor */
+#define CG_FORMAT_VERSION_ADJACENT 2 /* deltas to the previous token (cg_encode_adjacent) */
 #define CG_MAGIC 0x314B4743u /* bytes "CGK1" */
 #define CG_GROUP 10
 #define CG_PROB_BITS 12
@@ -251,6 +252,73 @@ cg_status cg_decode_into_paged(const cg_shape* shape, const uint8_t* in_dev, uin
                                uint16_t* pool_dev, int32_t num_pages, int32_t page_tokens,
                                const int32_t* block_table_dev, int64_t total_tokens,
                                int32_t* status_dev, cudaStream_t stream);
+
+/* Format 2: deltas between adjacent tokens.  [Practice] 1 describes the
+ * deltas as differences between adjacent tokens; format 1 (every call above)
+ * takes them against the group's reconstructed anchor so that every token
+ * decodes on its own.  Format 2 takes the page literally: inside a group,
+ * token t is quantised against the reconstruction of token t - 1,
+ *     q_t = clamp(roundf((x_t - x^_(t-1)) / step), -127, 127),
+ *     x^_t = x^_(t-1) + (float)q_t * step      (x^ of the anchor = a),
+ * each operation fp32 and rounded to nearest, no fused multiply-add; the chain
+ * restarts at every anchor, so a value depends on at most nine earlier ones.
+ * Anchors, tables, streams and the container layout are those of format 1;
+ * the header's version field is CG_FORMAT_VERSION_ADJACENT.  A format-2
+ * container given to a format-1 decoder, or the other way round, is
+ * CG_ERR_MISMATCH. */
+
+/* cg_encode writing format 2.  Arguments as cg_encode without tables_dev (the
+ * tables are always built from the format-2 symbols); the workspace is
+ * cg_encode_workspace_bytes. */
+cg_status cg_encode_adjacent(const cg_shape* shape, const uint16_t* kv_dev, int64_t total_tokens,
+                             int64_t token_start, int32_t num_chunks, int32_t chunk_tokens,
+                             cg_level level, uint8_t* out_dev, uint64_t out_stride,
+                             uint64_t* out_sizes_dev, int32_t* status_dev, void* workspace_dev,
+                             uint64_t workspace_bytes, cudaStream_t stream);
+
+/* cg_decode of format-2 containers (same arguments and layout).  Two launches:
+ * the rANS pass leaves every value's symbol (u16) in its destination slot,
+ * then a second kernel rebuilds each group's chain in place.  As in every
+ * decode call, a slot whose chunk or stream is reported corrupt holds
+ * undefined values. */
+cg_status cg_decode_adjacent(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
+                             int32_t num_chunks, int32_t chunk_tokens, cg_level level,
+                             uint16_t* out_dev, uint64_t out_elems, int32_t* status_dev,
+                             cudaStream_t stream);
+
+/* cg_decode_into of format-2 containers (same arguments, same two passes). */
+cg_status cg_decode_adjacent_into(const cg_shape* shape, const uint8_t* in_dev,
+                                  uint64_t in_stride, int32_t num_chunks, int32_t chunk_tokens,
+                                  cg_level level, uint16_t* kv_dev, int64_t total_tokens,
+                                  int32_t* status_dev, cudaStream_t stream);
+
+/* Device workspace cg_encode_levels needs for `num_chunks` chunks of
+ * `chunk_tokens` (about three times the symbol part of cg_encode's).  Host,
+ * pure. */
+cg_status cg_encode_levels_workspace_bytes(const cg_shape* shape, int32_t chunk_tokens,
+                                           int32_t num_chunks, uint64_t* bytes);
+
+/* Encode `num_chunks` consecutive chunks (the token ranges of cg_encode) at
+ * all three levels from one read of the fp16 cache.  Grounding: [Practice]
+ * 2.1 prepares three versions of every chunk ahead of sending, so that the
+ * sender can choose one per chunk as the bandwidth changes ([Practice] 2.2).
+ * The anchor range, the anchor codes and the reconstructed anchors do not
+ * depend on the level and are computed once; every delta is quantised at the
+ * three levels' steps in the same pass, and each level's histograms, tables
+ * and streams are then built as in cg_encode.
+ * Output: the container of (level j, chunk k) -- j = CG_LEVEL_HIGH,
+ * CG_LEVEL_BALANCED, CG_LEVEL_FAST -- goes to
+ * out_dev + (j*num_chunks + k)*out_stride and its size to
+ * out_sizes_dev[j*num_chunks + k] (u64, device); it is byte for byte the
+ * container cg_encode writes for that chunk at level j.  Tables are always
+ * built from the data.  The workspace (cg_encode_levels_workspace_bytes,
+ * 256-byte aligned) is the caller's, as for cg_encode.  Data errors:
+ * CG_ERR_NONFINITE, CG_ERR_CAPACITY (per container, as cg_encode). */
+cg_status cg_encode_levels(const cg_shape* shape, const uint16_t* kv_dev, int64_t total_tokens,
+                           int64_t token_start, int32_t num_chunks, int32_t chunk_tokens,
+                           uint8_t* out_dev, uint64_t out_stride, uint64_t* out_sizes_dev,
+                           int32_t* status_dev, void* workspace_dev, uint64_t workspace_bytes,
+                           cudaStream_t stream);
 
 /* cg_encode without caller-provided scratch.  The pages have no counterpart
  * to this call; it exists for callers that cannot allocate device memory --

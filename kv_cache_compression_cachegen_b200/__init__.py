@@ -18,7 +18,8 @@ __all__ = [
     "CG_ERR_NONFINITE", "CG_ERR_CUDA", "CG_ERR_UNSUPPORTED", "LEVELS", "CacheGenError",
     "Shape", "library", "library_path", "check", "cg_status_string", "cg_section_offsets",
     "cg_encoded_bound", "cg_tables_bytes", "cg_encode_workspace_bytes", "cg_build_tables",
-    "cg_encode", "cg_encode_static", "cg_decode", "cg_decode_into", "cg_decode_into_paged",
+    "cg_encode", "cg_encode_static", "cg_encode_levels", "cg_encode_levels_workspace_bytes",
+    "cg_encode_adjacent", "cg_decode_adjacent", "cg_decode_adjacent_into", "cg_decode", "cg_decode_into", "cg_decode_into_paged",
 ]
 
 CG_OK, CG_ERR_INVALID_ARG, CG_ERR_CAPACITY, CG_ERR_CORRUPT = 0, 1, 2, 3
@@ -71,6 +72,22 @@ _SIGNATURES = {
     "cg_encode_static": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_int64,
                                         ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                         ctypes.c_int, _P, _P, ctypes.c_uint64, _P, _P, _P]),
+    "cg_encode_levels_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(Shape), ctypes.c_int32,
+                                                        ctypes.c_int32,
+                                                        ctypes.POINTER(ctypes.c_uint64)]),
+    "cg_encode_levels": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P,
+                                        ctypes.c_uint64, _P, _P, _P, ctypes.c_uint64, _P]),
+    "cg_encode_adjacent": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_int64,
+                                          ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.c_int, _P, ctypes.c_uint64, _P, _P, _P,
+                                          ctypes.c_uint64, _P]),
+    "cg_decode_adjacent": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_uint64,
+                                          ctypes.c_int32, ctypes.c_int32, ctypes.c_int, _P,
+                                          ctypes.c_uint64, _P, _P]),
+    "cg_decode_adjacent_into": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_uint64,
+                                               ctypes.c_int32, ctypes.c_int32, ctypes.c_int, _P,
+                                               ctypes.c_int64, _P, _P]),
     "cg_decode": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_uint64, ctypes.c_int32,
                                  ctypes.c_int32, ctypes.c_int, _P, ctypes.c_uint64, _P, _P]),
     "cg_decode_into": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_uint64,
@@ -186,6 +203,46 @@ def cg_encode_static(shape, kv, total_tokens: int, token_start: int, num_chunks:
                                       token_start, num_chunks, chunk_tokens, int(level),
                                       _ptr(tables), _ptr(out), out_stride, _ptr(out_sizes),
                                       _ptr(status), _stream(stream))
+
+
+def cg_encode_levels_workspace_bytes(shape, chunk_tokens: int, num_chunks: int) -> int:
+    return _size_query("cg_encode_levels_workspace_bytes", ctypes.byref(_shape(shape)),
+                       chunk_tokens, num_chunks)
+
+
+def cg_encode_levels(shape, kv, total_tokens: int, token_start: int, num_chunks: int,
+                     chunk_tokens: int, out, out_stride: int, out_sizes, status, workspace,
+                     workspace_bytes: int, stream=None) -> int:
+    """All three levels from one quantiser pass; container (level j, chunk k)
+    at out + (j * num_chunks + k) * out_stride."""
+    return library().cg_encode_levels(ctypes.byref(_shape(shape)), _ptr(kv), total_tokens,
+                                      token_start, num_chunks, chunk_tokens, _ptr(out),
+                                      out_stride, _ptr(out_sizes), _ptr(status),
+                                      _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def cg_encode_adjacent(shape, kv, total_tokens: int, token_start: int, num_chunks: int,
+                       chunk_tokens: int, level: int, out, out_stride: int, out_sizes, status,
+                       workspace, workspace_bytes: int, stream=None) -> int:
+    """cg_encode writing format 2 (deltas between adjacent tokens)."""
+    return library().cg_encode_adjacent(ctypes.byref(_shape(shape)), _ptr(kv), total_tokens,
+                                        token_start, num_chunks, chunk_tokens, int(level),
+                                        _ptr(out), out_stride, _ptr(out_sizes), _ptr(status),
+                                        _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def cg_decode_adjacent(shape, inp, in_stride: int, num_chunks: int, chunk_tokens: int,
+                       level: int, out, out_elems: int, status, stream=None) -> int:
+    return library().cg_decode_adjacent(ctypes.byref(_shape(shape)), _ptr(inp), in_stride,
+                                        num_chunks, chunk_tokens, int(level), _ptr(out),
+                                        out_elems, _ptr(status), _stream(stream))
+
+
+def cg_decode_adjacent_into(shape, inp, in_stride: int, num_chunks: int, chunk_tokens: int,
+                            level: int, kv, total_tokens: int, status, stream=None) -> int:
+    return library().cg_decode_adjacent_into(ctypes.byref(_shape(shape)), _ptr(inp), in_stride,
+                                             num_chunks, chunk_tokens, int(level), _ptr(kv),
+                                             total_tokens, _ptr(status), _stream(stream))
 
 
 def cg_decode(shape, inp, in_stride: int, num_chunks: int, chunk_tokens: int, level: int, out,

@@ -165,11 +165,12 @@ cg_status cg_build_tables(const cg_shape* shape, const uint16_t* kv_dev, int64_t
   return from_cuda(cg::launch_encode(p, true, stream));
 }
 
-cg_status cg_encode(const cg_shape* shape, const uint16_t* kv_dev, int64_t total_tokens,
-                    int64_t token_start, int32_t num_chunks, int32_t chunk_tokens,
-                    cg_level level, const uint8_t* tables_dev, uint8_t* out_dev,
-                    uint64_t out_stride, uint64_t* out_sizes_dev, int32_t* status_dev,
-                    void* workspace_dev, uint64_t workspace_bytes, cudaStream_t stream) {
+static cg_status encode_common(const cg_shape* shape, const uint16_t* kv_dev,
+                               int64_t total_tokens, int64_t token_start, int32_t num_chunks,
+                               int32_t chunk_tokens, cg_level level, const uint8_t* tables_dev,
+                               uint8_t* out_dev, uint64_t out_stride, uint64_t* out_sizes_dev,
+                               int32_t* status_dev, void* workspace_dev,
+                               uint64_t workspace_bytes, int adjacent, cudaStream_t stream) {
   cg_status st =
       check_encode_args(shape, kv_dev, total_tokens, token_start, num_chunks, chunk_tokens, level);
   if (st != CG_OK) return st;
@@ -197,6 +198,7 @@ cg_status cg_encode(const cg_shape* shape, const uint16_t* kv_dev, int64_t total
   p.H = H;
   p.D = D;
   p.level = int(level);
+  p.adjacent = adjacent;
   p.out = out_dev;
   p.out_stride = out_stride;
   p.out_sizes = out_sizes_dev;
@@ -211,13 +213,86 @@ cg_status cg_encode(const cg_shape* shape, const uint16_t* kv_dev, int64_t total
   return from_cuda(cg::launch_encode(p, false, stream));
 }
 
+cg_status cg_encode(const cg_shape* shape, const uint16_t* kv_dev, int64_t total_tokens,
+                    int64_t token_start, int32_t num_chunks, int32_t chunk_tokens,
+                    cg_level level, const uint8_t* tables_dev, uint8_t* out_dev,
+                    uint64_t out_stride, uint64_t* out_sizes_dev, int32_t* status_dev,
+                    void* workspace_dev, uint64_t workspace_bytes, cudaStream_t stream) {
+  return encode_common(shape, kv_dev, total_tokens, token_start, num_chunks, chunk_tokens, level,
+                       tables_dev, out_dev, out_stride, out_sizes_dev, status_dev, workspace_dev,
+                       workspace_bytes, 0, stream);
+}
+
+cg_status cg_encode_adjacent(const cg_shape* shape, const uint16_t* kv_dev, int64_t total_tokens,
+                             int64_t token_start, int32_t num_chunks, int32_t chunk_tokens,
+                             cg_level level, uint8_t* out_dev, uint64_t out_stride,
+                             uint64_t* out_sizes_dev, int32_t* status_dev, void* workspace_dev,
+                             uint64_t workspace_bytes, cudaStream_t stream) {
+  return encode_common(shape, kv_dev, total_tokens, token_start, num_chunks, chunk_tokens, level,
+                       nullptr, out_dev, out_stride, out_sizes_dev, status_dev, workspace_dev,
+                       workspace_bytes, 1, stream);
+}
+
+cg_status cg_encode_levels_workspace_bytes(const cg_shape* shape, int32_t chunk_tokens,
+                                           int32_t num_chunks, uint64_t* bytes) {
+  cg_status st = check_shape(shape);
+  if (st != CG_OK) return st;
+  if ((st = check_chunk(shape, chunk_tokens)) != CG_OK) return st;
+  if (bytes == nullptr || num_chunks < 1) return CG_ERR_INVALID_ARG;
+  *bytes = cg::enc_levels_workspace(shape->num_layers, shape->num_kv_heads, shape->head_dim,
+                                    chunk_tokens, num_chunks)
+               .total;
+  return CG_OK;
+}
+
+cg_status cg_encode_levels(const cg_shape* shape, const uint16_t* kv_dev, int64_t total_tokens,
+                           int64_t token_start, int32_t num_chunks, int32_t chunk_tokens,
+                           uint8_t* out_dev, uint64_t out_stride, uint64_t* out_sizes_dev,
+                           int32_t* status_dev, void* workspace_dev, uint64_t workspace_bytes,
+                           cudaStream_t stream) {
+  cg_status st = check_encode_args(shape, kv_dev, total_tokens, token_start, num_chunks,
+                                   chunk_tokens, CG_LEVEL_BALANCED);
+  if (st != CG_OK) return st;
+  const int L = shape->num_layers, H = shape->num_kv_heads, D = shape->head_dim;
+  if (out_dev == nullptr || !aligned16(out_dev) || out_sizes_dev == nullptr ||
+      status_dev == nullptr || workspace_dev == nullptr || (out_stride % 16) != 0)
+    return CG_ERR_INVALID_ARG;
+  if (out_stride < cg::sections(L, H, D, chunk_tokens).payload) return CG_ERR_CAPACITY;
+  const cg::EncLevelsWorkspace ws = cg::enc_levels_workspace(L, H, D, chunk_tokens, num_chunks);
+  if (workspace_bytes < ws.total || (reinterpret_cast<uintptr_t>(workspace_dev) & 255u) != 0)
+    return workspace_bytes < ws.total ? CG_ERR_CAPACITY : CG_ERR_INVALID_ARG;
+  uint8_t* w = static_cast<uint8_t*>(workspace_dev);
+  cg::EncParams p{};
+  p.kv = kv_dev;
+  p.T = total_tokens;
+  p.token_start = token_start;
+  p.num_chunks = num_chunks;
+  p.C = chunk_tokens;
+  p.L = L;
+  p.H = H;
+  p.D = D;
+  p.level = CG_LEVEL_HIGH;
+  p.out_stride = out_stride;
+  p.lens = reinterpret_cast<uint32_t*>(w + ws.base.lens);
+  p.scratch = w + ws.base.scratch;
+  p.status = status_dev;
+  for (int j = 0; j < 3; ++j) {
+    p.lsym[j] = w + ws.sym[j];
+    p.letab[j] = reinterpret_cast<uint32_t*>(w + ws.etab[j]);
+    p.lslabtot[j] = reinterpret_cast<uint32_t*>(w + ws.slabtot[j]);
+    p.lout[j] = out_dev + uint64_t(j) * num_chunks * out_stride;
+  }
+  return from_cuda(cg::launch_encode_levels(p, out_sizes_dev, stream));
+}
+
 static cg_status decode_common(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
                                int32_t num_chunks, int32_t chunk_tokens, cg_level level,
                                uint16_t* out_dev, uint64_t out_elems, int into,
                                int64_t total_tokens, int32_t* status_dev, cudaStream_t stream,
                                const int32_t* block_table = nullptr, int32_t num_pages = 0,
-                               int32_t page_tokens = 0) {
+                               int32_t page_tokens = 0, int adjacent = 0) {
   cg::DecParams p{};
+  p.adjacent = adjacent;
   p.block_table = block_table;
   p.num_pages = num_pages;
   p.page_tokens = page_tokens;
@@ -263,6 +338,47 @@ cg_status cg_decode_into(const cg_shape* shape, const uint8_t* in_dev, uint64_t 
                          shape->num_kv_heads * shape->head_dim;
   return decode_common(shape, in_dev, in_stride, num_chunks, chunk_tokens, level, kv_dev, elems,
                        1, total_tokens, status_dev, stream);
+}
+
+// Format 2 decodes in two launches: the rANS pass leaves the symbols in the
+// destination, then chain_kernel rebuilds the values (one CTA of 256 threads
+// per 256 (group, 8-channel block) pairs of a (chunk, layer, K/V)).
+static cg_status check_chain_grid(const cg_shape* shape, int32_t num_chunks,
+                                  int32_t chunk_tokens) {
+  const uint64_t work = uint64_t((chunk_tokens + CG_GROUP - 1) / CG_GROUP) *
+                        (uint64_t(shape->num_kv_heads) * shape->head_dim / 8);
+  const uint64_t blocks = uint64_t(num_chunks) * shape->num_layers * 2 * ((work + 255) / 256);
+  return blocks > 0x7FFFFFFFull ? CG_ERR_UNSUPPORTED : CG_OK;
+}
+
+cg_status cg_decode_adjacent(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
+                             int32_t num_chunks, int32_t chunk_tokens, cg_level level,
+                             uint16_t* out_dev, uint64_t out_elems, int32_t* status_dev,
+                             cudaStream_t stream) {
+  cg_status st = check_decode_args(shape, in_dev, in_stride, num_chunks, chunk_tokens, level,
+                                   out_dev, status_dev);
+  if (st != CG_OK) return st;
+  if ((st = check_chain_grid(shape, num_chunks, chunk_tokens)) != CG_OK) return st;
+  const uint64_t slot = uint64_t(shape->num_layers) * 2 * chunk_tokens * shape->num_kv_heads *
+                        shape->head_dim;
+  if (out_elems < slot * uint64_t(num_chunks)) return CG_ERR_CAPACITY;
+  return decode_common(shape, in_dev, in_stride, num_chunks, chunk_tokens, level, out_dev,
+                       out_elems, 0, 0, status_dev, stream, nullptr, 0, 0, 1);
+}
+
+cg_status cg_decode_adjacent_into(const cg_shape* shape, const uint8_t* in_dev,
+                                  uint64_t in_stride, int32_t num_chunks, int32_t chunk_tokens,
+                                  cg_level level, uint16_t* kv_dev, int64_t total_tokens,
+                                  int32_t* status_dev, cudaStream_t stream) {
+  cg_status st = check_decode_args(shape, in_dev, in_stride, num_chunks, chunk_tokens, level,
+                                   kv_dev, status_dev);
+  if (st != CG_OK) return st;
+  if ((st = check_chain_grid(shape, num_chunks, chunk_tokens)) != CG_OK) return st;
+  if (total_tokens < 1) return CG_ERR_INVALID_ARG;
+  const uint64_t elems = uint64_t(shape->num_layers) * 2 * uint64_t(total_tokens) *
+                         shape->num_kv_heads * shape->head_dim;
+  return decode_common(shape, in_dev, in_stride, num_chunks, chunk_tokens, level, kv_dev, elems,
+                       1, total_tokens, status_dev, stream, nullptr, 0, 0, 1);
 }
 
 cg_status cg_decode_into_paged(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,

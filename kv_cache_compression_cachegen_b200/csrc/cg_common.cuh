@@ -106,6 +106,36 @@ __host__ __device__ inline EncWorkspace enc_workspace(int L, int H, int D, int C
   return w;
 }
 
+// Workspace of the three-level encoder (cg_encode_levels): one encoder
+// workspace whose stream lengths and word slots the three levels reuse in
+// turn, plus a symbol array, constants and word totals for each level.
+struct EncLevelsWorkspace {
+  EncWorkspace base;  // level 0's symbols, constants and totals; shared lens and scratch
+  uint64_t sym[3], etab[3], slabtot[3];
+  uint64_t total;
+};
+
+__host__ __device__ inline EncLevelsWorkspace enc_levels_workspace(int L, int H, int D, int C,
+                                                                   int chunks) {
+  EncLevelsWorkspace w;
+  w.base = enc_workspace(L, H, D, C, chunks);
+  w.sym[0] = w.base.sym;
+  w.etab[0] = w.base.etab;
+  w.slabtot[0] = w.base.slabtot;
+  const uint64_t streams = uint64_t(chunks) * L * 2 * C;
+  uint64_t at = w.base.total;
+  for (int k = 1; k < 3; ++k) {
+    w.sym[k] = at;
+    at = up256(at + streams * uint64_t(H) * D);
+    w.etab[k] = at;
+    at = up256(at + uint64_t(chunks) * L * 2 * H * 256 * 16);
+    w.slabtot[k] = at;
+    at = up256(at + uint64_t(chunks) * L * 2 * 4);
+  }
+  w.total = at;
+  return w;
+}
+
 // Kernel launch parameters shared by the encoder kernels.
 struct EncParams {
   const uint16_t* kv;      // [L][2][T][H][D]
@@ -115,6 +145,7 @@ struct EncParams {
   int C;                   // nominal chunk size
   int L, H, D;
   int level;
+  int adjacent;            // 0: format 1 (deltas to the anchor); 1: format 2 (adjacent tokens)
   uint8_t* out;            // containers (null when only tables are built)
   uint64_t out_stride;
   uint64_t* out_sizes;     // [num_chunks]
@@ -127,6 +158,12 @@ struct EncParams {
   uint32_t* slabtot;
   uint8_t* scratch;
   int32_t* status;
+  // Three-level encode only (quant_kernel<3>): per level, its symbols,
+  // encoder constants, word totals and containers.
+  uint8_t* lsym[3];
+  uint32_t* letab[3];
+  uint32_t* lslabtot[3];
+  uint8_t* lout[3];
 };
 
 struct DecParams {
@@ -135,6 +172,7 @@ struct DecParams {
   int num_chunks;
   int C, L, H, D;
   int level;
+  int adjacent;            // 1: format 2 containers; decode writes codes, then rebuilds chains
   uint16_t* out;
   uint64_t out_elems;      // size of out in elements (checked against the shape by the C ABI)
   int into;                // 0: chunk slots [L][2][n][H][D]; 1: full KV [L][2][T][H][D];
@@ -149,6 +187,7 @@ struct DecParams {
 
 // Kernel launchers (encode.cu, decode.cu).
 cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stream);
+cudaError_t launch_encode_levels(const EncParams& p, uint64_t* out_sizes, cudaStream_t stream);
 cudaError_t launch_decode(const DecParams& p, cudaStream_t stream);
 
 }  // namespace cg

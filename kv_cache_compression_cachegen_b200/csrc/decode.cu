@@ -282,8 +282,15 @@ __device__ __forceinline__ void store16h(uint16_t* dst, const uint32_t (&hv)[8],
   }
 }
 
+// The symbol u = q + 127 of a packed slot entry (format 2's first pass stores
+// the symbols themselves, as u16, in the destination).
+__device__ __forceinline__ uint32_t pack_codes(uint32_t e0, uint32_t e1) {
+  return (e0 >> 24) | ((e1 >> 8) & 0x00FF0000u);
+}
+
 // Delta lane: decode head h of its stream in steps of 8 values; the values of
-// two steps leave as one 32-byte store.
+// two steps leave as one 32-byte store.  CODES: the symbols instead of values.
+template <bool CODES>
 __device__ __forceinline__ void decode_delta_head(uint32_t& x, Pos& ps, Ring& r,
                                                   const uint32_t* __restrict__ tbl, float step,
                                                   const float* __restrict__ arow,
@@ -303,10 +310,14 @@ __device__ __forceinline__ void decode_delta_head(uint32_t& x, Pos& ps, Ring& r,
 #pragma unroll
       for (int k = 0; k < 8; k += 2) {
         const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl);
-        const float v0 = __fadd_rn(a[k], __fmul_rn(sym_value(e0), step));
         const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl);
-        const float v1 = __fadd_rn(a[k + 1], __fmul_rn(sym_value(e1), step));
-        hv[4 * half + (k >> 1)] = pack_half2(v0, v1);
+        if constexpr (CODES) {
+          hv[4 * half + (k >> 1)] = pack_codes(e0, e1);
+        } else {
+          const float v0 = __fadd_rn(a[k], __fmul_rn(sym_value(e0), step));
+          const float v1 = __fadd_rn(a[k + 1], __fmul_rn(sym_value(e1), step));
+          hv[4 * half + (k >> 1)] = pack_half2(v0, v1);
+        }
       }
       ps.p += (ps.ra - ra0) >> 1;
     }
@@ -316,6 +327,8 @@ __device__ __forceinline__ void decode_delta_head(uint32_t& x, Pos& ps, Ring& r,
 
 // Anchor lane: decode head h, write fp16(a) and keep a (fp32) for the deltas.
 // zp and sc point at the head's zero points and scales staged in shared memory.
+// CODES: store the symbols only (format 2 rebuilds the values afterwards).
+template <bool CODES>
 __device__ __forceinline__ void decode_anchor_head(uint32_t& x, Pos& ps, Ring& r,
                                                    const uint32_t* __restrict__ tbl,
                                                    const float* __restrict__ zp,
@@ -337,22 +350,82 @@ __device__ __forceinline__ void decode_anchor_head(uint32_t& x, Pos& ps, Ring& r
       const float4 s1 = *reinterpret_cast<const float4*>(sc + dd + 4);
       const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
       const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      float v[8];
+      if constexpr (CODES) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t e = rans_step(x, ps.ra, ps.w, tbl);
-        v[k] = __fadd_rn(z[k], __fmul_rn(sym_value(e), s[k]));
+        for (int k = 0; k < 8; k += 2) {
+          const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl);
+          const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl);
+          hv[4 * half + (k >> 1)] = pack_codes(e0, e1);
+        }
+        ps.p += (ps.ra - ra0) >> 1;
+      } else {
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t e = rans_step(x, ps.ra, ps.w, tbl);
+          v[k] = __fadd_rn(z[k], __fmul_rn(sym_value(e), s[k]));
+        }
+        ps.p += (ps.ra - ra0) >> 1;
+        *reinterpret_cast<float4*>(arow + dd) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4*>(arow + dd + 4) = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) hv[4 * half + k] = pack_half2(v[2 * k], v[2 * k + 1]);
       }
-      ps.p += (ps.ra - ra0) >> 1;
-      *reinterpret_cast<float4*>(arow + dd) = make_float4(v[0], v[1], v[2], v[3]);
-      *reinterpret_cast<float4*>(arow + dd + 4) = make_float4(v[4], v[5], v[6], v[7]);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) hv[4 * half + k] = pack_half2(v[2 * k], v[2 * k + 1]);
     }
     store16h(orow + d0, hv, al32);
   }
 }
 
+// Header validation of one container (both decode kernels run it; every CTA
+// of a chunk checks the same 64 bytes).  Returns 0 or the status to report.
+__device__ int check_header(const uint8_t* base, const DecParams& p, cg_header& h) {
+  const uint4* hp = reinterpret_cast<const uint4*>(base);
+  uint4* hd = reinterpret_cast<uint4*>(&h);
+  for (int i = 0; i < 4; ++i) hd[i] = __ldg(hp + i);
+  const int L = p.L, H = p.H, D = p.D;
+  const uint32_t want = p.adjacent ? CG_FORMAT_VERSION_ADJACENT : CG_FORMAT_VERSION;
+  int err = 0;
+  if (h.magic != CG_MAGIC || h.group != kGroup || h.prob_bits != kProbBits || h.reserved != 0 ||
+      (h.version != CG_FORMAT_VERSION && h.version != CG_FORMAT_VERSION_ADJACENT))
+    err = CG_ERR_CORRUPT;
+  else if (h.version != want || h.level != uint32_t(p.level) ||
+           h.num_layers != uint32_t(L) || h.num_kv_heads != uint32_t(H) ||
+           h.head_dim != uint32_t(D) || h.chunk_tokens != uint32_t(p.C))
+    err = CG_ERR_MISMATCH;  // the other format, or another level or shape
+  else if (h.n_tokens < 1 || h.n_tokens > uint32_t(p.C))
+    err = CG_ERR_CORRUPT;
+  if (!err) {
+    const Sections sec = sections(L, H, D, h.n_tokens);
+    if (h.payload_bytes > 0xFFFFFFFFull || h.total_bytes > p.in_stride ||
+        sec.payload + h.payload_bytes > h.total_bytes ||
+        up16(sec.payload + h.payload_bytes) != h.total_bytes)
+      err = CG_ERR_CORRUPT;
+    else if (p.into && (h.token_start > uint64_t(p.total_tokens) ||
+                        h.token_start + h.n_tokens > uint64_t(p.total_tokens)))
+      err = CG_ERR_MISMATCH;
+  }
+  return err;
+}
+
+// Destination row (H*D values) of local token t of a chunk, or null when a
+// paged destination's block table does not map it.
+__device__ __forceinline__ uint16_t* dest_row(const DecParams& p, int chunk, int slab, int n,
+                                              long long tstart, int t) {
+  const int H = p.H, D = p.D;
+  if (p.into == 1)
+    return p.out + ((uint64_t(slab) * p.total_tokens + uint64_t(tstart) + t) * H) * D;
+  if (p.into == 2) {
+    const int64_t g = tstart + t;  // logical token g: row g mod P of page block_table[g / P]
+    const int32_t page = __ldg(p.block_table + g / p.page_tokens);
+    if (page < 0 || page >= p.num_pages) return nullptr;
+    return p.out + (((uint64_t(slab) * p.num_pages + uint64_t(page)) * p.page_tokens +
+                     uint64_t(g % p.page_tokens)) * H) * D;
+  }
+  return p.out + uint64_t(chunk) * (uint64_t(p.L) * 2 * p.C * H * D) +
+         ((uint64_t(slab) * n + t) * H) * D;
+}
+
+template <bool CODES>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_ok, s_n, s_bad;
@@ -370,31 +443,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   const uint8_t* base = p.in + uint64_t(chunk) * p.in_stride;
 
   if (tid == 0) {
-    // Header validation (every CTA of the chunk checks the same 64 bytes).
-    const uint4* hp = reinterpret_cast<const uint4*>(base);
     cg_header h;
-    uint4* hd = reinterpret_cast<uint4*>(&h);
-    for (int i = 0; i < 4; ++i) hd[i] = __ldg(hp + i);
-    int err = 0;
-    if (h.magic != CG_MAGIC || h.version != CG_FORMAT_VERSION || h.group != kGroup ||
-        h.prob_bits != kProbBits || h.reserved != 0)
-      err = CG_ERR_CORRUPT;
-    else if (h.level != uint32_t(p.level) || h.num_layers != uint32_t(L) ||
-             h.num_kv_heads != uint32_t(H) || h.head_dim != uint32_t(D) ||
-             h.chunk_tokens != uint32_t(p.C))
-      err = CG_ERR_MISMATCH;
-    else if (h.n_tokens < 1 || h.n_tokens > uint32_t(p.C))
-      err = CG_ERR_CORRUPT;
-    if (!err) {
-      const Sections sec = sections(L, H, D, h.n_tokens);
-      if (h.payload_bytes > 0xFFFFFFFFull || h.total_bytes > p.in_stride ||
-          sec.payload + h.payload_bytes > h.total_bytes ||
-          up16(sec.payload + h.payload_bytes) != h.total_bytes)
-        err = CG_ERR_CORRUPT;
-      else if (p.into && (h.token_start > uint64_t(p.total_tokens) ||
-                          h.token_start + h.n_tokens > uint64_t(p.total_tokens)))
-        err = CG_ERR_MISMATCH;
-    }
+    const int err = check_header(base, p, h);
     if (err) set_status(p.status, err);
     s_ok = !err;
     s_n = int(h.n_tokens);
@@ -467,24 +517,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   }
   bool active = token < n;
   const uint32_t* offs = reinterpret_cast<const uint32_t*>(base + sec.offsets);
-  // Destination row of this thread's token.
+  // Destination row of this thread's token (a paged pool's block table may
+  // leave it unmapped: nothing is written for it).
   uint16_t* orow = p.out;
-  if (p.into == 1) {
-    orow = p.out + ((uint64_t(slab) * p.total_tokens + uint64_t(s_tstart) + token) * H) * D;
-  } else if (p.into == 2) {
-    // paged pool: logical token t is row t mod P of page block_table[t / P]
-    const int64_t t = s_tstart + token;
-    const int32_t page = active ? __ldg(p.block_table + t / p.page_tokens) : 0;
-    if (page < 0 || page >= p.num_pages) {
+  if (active) {
+    orow = dest_row(p, chunk, slab, n, s_tstart, token);
+    if (orow == nullptr) {
       set_status(p.status, CG_ERR_MISMATCH);
       active = false;
-    } else {
-      orow = p.out + (((uint64_t(slab) * p.num_pages + uint64_t(page)) * p.page_tokens +
-                       uint64_t(t % p.page_tokens)) * H) * D;
+      orow = p.out;
     }
-  } else {
-    orow = p.out + uint64_t(chunk) * (uint64_t(L) * 2 * p.C * H * D) +
-           ((uint64_t(slab) * n + token) * H) * D;
   }
   Ring ring;
   ring.gbase = base;
@@ -549,7 +591,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
         float* arow = ahat + ((h & 1) * kUnitGroups + g_local) * astride;
         const float* zh = zs + (h & 1) * 2 * D;
         const int one = single[h];
-        if (one >= 0) {
+        if (one >= 0 && CODES) {
+          const uint32_t cc = uint32_t(one) * 0x10001u;
+          for (int d0 = 0; d0 < D; d0 += 8)
+            *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(cc, cc, cc, cc);
+        } else if (one >= 0) {
           const float c = float(one - 127);
           for (int d0 = 0; d0 < D; d0 += 8) {
             float v[8];
@@ -562,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
                            pack_half2(v[4], v[5]), pack_half2(v[6], v[7]));
           }
         } else {
-          decode_anchor_head(x, ps, ring, tb, zh, zh + D, arow, orow + h * D, D, al32);
+          decode_anchor_head<CODES>(x, ps, ring, tb, zh, zh + D, arow, orow + h * D, D, al32);
         }
       }
     } else if (it >= 1 && active) {
@@ -570,7 +616,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
       const uint32_t* tb = tbl + (h % 3) * kM;
       const float* arow = ahat + ((h & 1) * kUnitGroups + g_local) * astride;
       const int one = single[h];
-      if (one >= 0) {
+      if (one >= 0 && CODES) {
+        const uint32_t cc = uint32_t(one) * 0x10001u;
+        for (int d0 = 0; d0 < D; d0 += 8)
+          *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(cc, cc, cc, cc);
+      } else if (one >= 0) {
         const float v = __fmul_rn(float(one - 127), step);
         for (int d0 = 0; d0 < D; d0 += 8) {
           uint32_t hv[4];
@@ -580,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
           *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
       } else {
-        decode_delta_head(x, ps, ring, tb, step, arow, orow + h * D, D, al32);
+        decode_delta_head<CODES>(x, ps, ring, tb, step, arow, orow + h * D, D, al32);
       }
     }
     if (scan_warp) cum_compact(fq, cum_buf(cumb + (it & 1) * kCumBuf), lane);
@@ -598,15 +648,90 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   if (active && (x != kRansL || ps.p != pend)) set_status(p.status, CG_ERR_CORRUPT);
 }
 
+// ---- format 2, second pass -------------------------------------------------
+// decode_kernel<true> has left every value's symbol u = q + 127 (a u16) in its
+// destination slot.  One thread per (anchor group, 8 channels of the token
+// row) rebuilds the group's chain in place: the anchor a = zp + c * scale,
+// then x^_t = x^_(t-1) + q_t * step for the group's later tokens, each sum and
+// product rounded to nearest (no contraction), each value stored as fp16.  The
+// ten rows' symbols are loaded before the first store, so a thread keeps ten
+// 16-byte loads in flight; a warp covers 512 contiguous bytes of each row.
+constexpr int kChainThreads = 256;
+
+__global__ void __launch_bounds__(kChainThreads) chain_kernel(const DecParams p,
+                                                              const int blocks_per_slab) {
+  __shared__ int s_ok, s_n;
+  __shared__ long long s_tstart;
+  const int tid = threadIdx.x;
+  const int part = blockIdx.x % blocks_per_slab;
+  const int rest = blockIdx.x / blocks_per_slab;
+  const int slab = rest % (2 * p.L);
+  const int chunk = rest / (2 * p.L);
+  const int L = p.L, H = p.H, D = p.D;
+  const uint8_t* base = p.in + uint64_t(chunk) * p.in_stride;
+  if (tid == 0) {
+    cg_header h;
+    s_ok = check_header(base, p, h) == 0;  // the decode pass has reported any error
+    s_n = int(h.n_tokens);
+    s_tstart = (long long)h.token_start;
+  }
+  __syncthreads();
+  if (!s_ok) return;
+  const int n = s_n;
+  const int rb = H * D / 8;  // 8-channel blocks of a token row
+  const int64_t w = int64_t(part) * kChainThreads + tid;
+  if (w >= int64_t((n + kGroup - 1) / kGroup) * rb) return;
+  const int g = int(w / rb), c0 = int(w % rb) * 8;
+  const int t0 = g * kGroup, ntok = min(kGroup, n - t0);
+  const Sections sec = sections(L, H, D, n);
+  const float* zp = reinterpret_cast<const float*>(base + sec.zp) + uint64_t(slab) * H * D + c0;
+  const float* sc = reinterpret_cast<const float*>(base + sec.scale) + uint64_t(slab) * H * D + c0;
+  const float4 z0 = __ldg(reinterpret_cast<const float4*>(zp));
+  const float4 z1 = __ldg(reinterpret_cast<const float4*>(zp + 4));
+  const float4 s0 = __ldg(reinterpret_cast<const float4*>(sc));
+  const float4 s1 = __ldg(reinterpret_cast<const float4*>(sc + 4));
+  const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+  const float sa[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  const float step = step_of(p.level, slab >> 1, L);
+
+  uint16_t* rows[kGroup];
+  uint4 cv[kGroup];
+#pragma unroll
+  for (int r = 0; r < kGroup; ++r) {
+    rows[r] = r < ntok ? dest_row(p, chunk, slab, n, s_tstart, t0 + r) : nullptr;
+    cv[r] = rows[r] ? *reinterpret_cast<const uint4*>(rows[r] + c0) : make_uint4(0, 0, 0, 0);
+  }
+  float x[8];
+#pragma unroll
+  for (int r = 0; r < kGroup; ++r) {
+    if (rows[r] == nullptr) break;  // end of the chunk (or an unmapped page)
+    const uint32_t cw[4] = {cv[r].x, cv[r].y, cv[r].z, cv[r].w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float q = float(int((cw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu) - 127);
+      x[k] = r == 0 ? __fadd_rn(z[k], __fmul_rn(q, sa[k])) : __fadd_rn(x[k], __fmul_rn(q, step));
+    }
+    *reinterpret_cast<uint4*>(rows[r] + c0) =
+        make_uint4(pack_half2(x[0], x[1]), pack_half2(x[2], x[3]), pack_half2(x[4], x[5]),
+                   pack_half2(x[6], x[7]));
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const DecParams& p, cudaStream_t stream) {
   const DecSmem sm = dec_smem(p.H, p.D);
-  cudaError_t err = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(sm.total));
+  auto* kern = p.adjacent ? decode_kernel<true> : decode_kernel<false>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm.total));
   if (err != cudaSuccess) return err;
   const uint64_t blocks = uint64_t(p.num_chunks) * p.L * 2 * p.units_per_slab;
-  decode_kernel<<<unsigned(blocks), kThreads, sm.total, stream>>>(p);
+  kern<<<unsigned(blocks), kThreads, sm.total, stream>>>(p);
+  if ((err = cudaGetLastError()) != cudaSuccess || !p.adjacent) return err;
+  const uint64_t work = uint64_t((p.C + kGroup - 1) / kGroup) * (p.H * p.D / 8);
+  const int per_slab = int((work + kChainThreads - 1) / kChainThreads);
+  chain_kernel<<<unsigned(uint64_t(p.num_chunks) * p.L * 2 * per_slab), kChainThreads, 0,
+                 stream>>>(p, per_slab);
   return cudaGetLastError();
 }
 

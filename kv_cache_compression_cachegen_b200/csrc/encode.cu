@@ -12,7 +12,10 @@
 //   quant_kernel    one CTA per (chunk, l, kv, h): anchor range -> zp, scale;
 //                   anchor codes and reconstructed anchors; delta symbols;
 //                   lane-replicated shared histogram; frequency table and the
-//                   encoder's per-symbol division constants.
+//                   encoder's per-symbol division constants.  quant_kernel<3>
+//                   (cg_encode_levels) quantises every delta at the three
+//                   levels' steps from one read and keeps three histograms;
+//                   the three kernels below then run once per level.
 //   rans_kernel     one thread per stream (l, kv, t), symbols in reverse;
 //                   renormalisation words go through a per-thread ring in
 //                   shared memory and leave in 32-byte blocks, written
@@ -39,27 +42,38 @@ constexpr int kScanThreads = 256;
 
 enum QuantMode { kModeEncode = 0, kModeTablesOnly = 1, kModeSuppliedTables = 2 };
 
+// Shared memory of quant_kernel<NL> (NL = levels quantised at once: 1, or 3
+// for the three-level encoder).
 struct QSmem {
-  uint32_t hist;    // u32 [255][32]  lane-replicated counters (bank = lane)
+  uint32_t hist;    // u32 [NL][255][32]  lane-replicated counters (bank = lane)
   uint32_t zp;      // f32 [256]
   uint32_t sc;      // f32 [256]
   uint32_t rcp;     // f32 [256]
   uint32_t red;     // f32 [2][8 warps][256]  anchor range partials (phase A)
-  uint32_t counts;  // u32 [256]  histogram totals (phase C, aliases red)
+  uint32_t counts;  // u32 [NL][256]  histogram totals (phase C)
   uint32_t total;
 };
 
 __host__ __device__ inline uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
 
+template <int NL>
 __host__ __device__ inline QSmem q_smem() {
   QSmem s;
   s.hist = 0;
-  s.zp = a16(s.hist + 255u * 32u * 4u);
+  s.zp = a16(s.hist + NL * 255u * 32u * 4u);
   s.sc = s.zp + 1024u;
   s.rcp = s.sc + 1024u;
-  s.red = s.rcp + 1024u;
-  s.counts = s.red;
-  s.total = a16(s.red + 2u * kQWarps * 256u * 4u);
+  if (NL == 1) {
+    s.red = s.rcp + 1024u;
+    s.counts = s.red;  // phase C reuses the phase-A partials
+    s.total = a16(s.red + 2u * kQWarps * 256u * 4u);
+  } else {
+    // The phase-A partials live in the histogram space, which is cleared
+    // after phase A; two CTAs per SM still fit.
+    s.red = s.hist;
+    s.counts = s.rcp + 1024u;
+    s.total = a16(s.counts + NL * 256u * 4u);
+  }
   return s;
 }
 
@@ -232,7 +246,19 @@ __device__ __forceinline__ void unpack8(const uint4 rv, float (&x)[8]) {
   }
 }
 
+// quant_kernel<NL, ADJ>: NL = 1 quantises at the call's level (cg_encode,
+// cg_build_tables); NL = 3 quantises every delta at the three levels' steps
+// from one read of the fp16 rows (cg_encode_levels: [Practice] 2.1 keeps three
+// versions of every chunk).  The anchor range, the anchor codes and the
+// reconstructed anchors do not depend on the level, so they are computed once
+// and the anchor codes enter every level's streams and histogram.
+// ADJ (format 2, cg_encode_adjacent): each delta is taken against the
+// reconstruction of the token before it ([Practice] 1: differences between
+// adjacent tokens) instead of the group's anchor; a lane walks its group's
+// rows in order, so the running reconstruction stays in its registers.
+template <int NL, bool ADJ>
 __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, const int mode) {
+  static_assert(!(ADJ && NL != 1), "format 2 is encoded one level at a time");
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int rest = blockIdx.x;
@@ -251,7 +277,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
   const uint64_t rs = uint64_t(H) * D;
   const uint16_t* col = p.kv + (uint64_t(slab) * p.T + t0) * rs + uint64_t(h) * D;
 
-  const QSmem sm = q_smem();
+  const QSmem sm = q_smem<NL>();
   uint32_t* hist = reinterpret_cast<uint32_t*>(smem + sm.hist);
   float* zp = reinterpret_cast<float*>(smem + sm.zp);
   float* sc = reinterpret_cast<float*>(smem + sm.sc);
@@ -260,7 +286,11 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
   uint32_t* counts = reinterpret_cast<uint32_t*>(smem + sm.counts);
 
   const Sections sec = sections(L, H, D, n);
-  uint8_t* cont = p.out ? p.out + uint64_t(chunk) * p.out_stride : nullptr;
+  // container of level j (of the call's level when NL == 1)
+  auto cont_of = [&](int j) -> uint8_t* {
+    uint8_t* o = NL == 1 ? p.out : p.lout[j];
+    return o ? o + uint64_t(chunk) * p.out_stride : nullptr;
+  };
   // Table block offsets equal container offsets minus the header.
   const uint64_t tb_zp = sec.zp - CG_HEADER_BYTES, tb_sc = sec.scale - CG_HEADER_BYTES,
                  tb_fq = sec.freq - CG_HEADER_BYTES;
@@ -270,9 +300,13 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
   const int ch = 8 * ql.c;  // first channel of this lane
   const int nsets = (Gn + ql.rpw - 1) / ql.rpw;
 
-  if (want_hist)
+  if (NL == 1 && want_hist)
     for (int i = tid; i < kAlphabet * 32; i += kQThreads) hist[i] = 0;
-  if (want_sym && h == 0 && tid == 0) p.slabtot[uint64_t(chunk) * L * 2 + slab] = 0;
+  if (want_sym && h == 0 && tid == 0) {
+#pragma unroll
+    for (int j = 0; j < NL; ++j)
+      (NL == 1 ? p.slabtot : p.lslabtot[j])[uint64_t(chunk) * L * 2 + slab] = 0;
+  }
 
   // ---- Phase A: per-channel anchor range -> zp, scale (or the supplied ones).
   bool nonfinite = false;
@@ -333,11 +367,17 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
     }
   }
   __syncthreads();
+  if (NL > 1 && want_hist)  // the phase-A partials are consumed: clear the histograms
+    for (int i = tid; i < NL * kAlphabet * 32; i += kQThreads) hist[i] = 0;
   for (int d = tid; d < D; d += kQThreads) {
     rcp[d] = sc[d] == 0.0f ? 0.0f : __frcp_rn(sc[d]);
-    if (cont) {
-      reinterpret_cast<float*>(cont + sec.zp)[uint64_t(tab) * D + d] = zp[d];
-      reinterpret_cast<float*>(cont + sec.scale)[uint64_t(tab) * D + d] = sc[d];
+#pragma unroll
+    for (int j = 0; j < NL; ++j) {
+      uint8_t* cont = cont_of(j);
+      if (cont) {
+        reinterpret_cast<float*>(cont + sec.zp)[uint64_t(tab) * D + d] = zp[d];
+        reinterpret_cast<float*>(cont + sec.scale)[uint64_t(tab) * D + d] = sc[d];
+      }
     }
     if (p.tables_out) {
       uint8_t* tb = p.tables_out + uint64_t(chunk) * p.tables_stride;
@@ -350,10 +390,25 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
   // ---- Phase B: quantise group by group.  Each lane loads the ten rows of its
   // group for its 8 channels; the rows of the warp's next group set are loaded
   // before the current set is quantised.
-  const float step = step_of(p.level, l, L);
-  const float rstep = __frcp_rn(step);
-  uint8_t* symc = p.sym + ((uint64_t(chunk) * L * 2 + slab) * H + h) * uint64_t(D / 16) * C * 16 +
-                  (ql.c >> 1) * uint64_t(C) * 16 + (ql.c & 1) * 8;
+  float step[NL], rstep[NL];
+#pragma unroll
+  for (int j = 0; j < NL; ++j) {
+    step[j] = step_of(NL == 1 ? p.level : j, l, L);
+    rstep[j] = __frcp_rn(step[j]);
+  }
+  const uint64_t symo = ((uint64_t(chunk) * L * 2 + slab) * H + h) * uint64_t(D / 16) * C * 16 +
+                        (ql.c >> 1) * uint64_t(C) * 16 + (ql.c & 1) * 8;
+  auto symc_of = [&](int j) { return (NL == 1 ? p.sym : p.lsym[j]) + symo; };
+  auto put_syms = [&](int j, int tok, const uint32_t (&u)[8]) {
+    if (want_hist) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) atomicAdd(&hist[(j * kAlphabet + u[k]) * 32 + lane], 1u);
+    }
+    if (want_sym)
+      *reinterpret_cast<uint2*>(symc_of(j) + uint64_t(tok) * 16) =
+          make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
+                     u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
+  };
   uint4 nx[kGroup];
   auto load_set = [&](int gs, uint4 (&v)[kGroup]) {
     const int g = gs * ql.rpw + ql.r;
@@ -397,54 +452,53 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
         if (!ok) u[k] = quant_exact(x[k], zc[k], scc[k]);
         a[k] = __fadd_rn(zc[k], __fmul_rn(float(int(u[k]) - 127), scc[k]));
       }
-      if (want_hist) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) atomicAdd(&hist[u[k] * 32 + lane], 1u);
-      }
-      if (want_sym)
-        *reinterpret_cast<uint2*>(symc + uint64_t(tg) * 16) =
-            make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
-                       u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
+      for (int j = 0; j < NL; ++j) put_syms(j, tg, u);
     }
 #pragma unroll
-    for (int j = 1; j < kGroup; ++j) {
-      if (j >= ntok) break;
+    for (int r = 1; r < kGroup; ++r) {
+      if (r >= ntok) break;
       float x[8];
-      unpack8(cur[j], x);
-      bool ok = true;
-      uint32_t u[8];
+      unpack8(cur[r], x);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) u[k] = quant_fast(__fsub_rn(x[k], a[k]), rstep, ok);
-      if (!ok) {
+      for (int j = 0; j < NL; ++j) {
+        bool ok = true;
+        uint32_t u[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (!isfinite(x[k])) nonfinite = true;
-          u[k] = quant_exact(x[k], a[k], step);
+        for (int k = 0; k < 8; ++k) u[k] = quant_fast(__fsub_rn(x[k], a[k]), rstep[j], ok);
+        if (!ok) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (!isfinite(x[k])) nonfinite = true;
+            u[k] = quant_exact(x[k], a[k], step[j]);
+          }
+        }
+        put_syms(j, tg + r, u);
+        if (ADJ) {  // the next row's reference: this row's reconstruction
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            a[k] = __fadd_rn(a[k], __fmul_rn(float(int(u[k]) - 127), step[j]));
         }
       }
-      if (want_hist) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) atomicAdd(&hist[u[k] * 32 + lane], 1u);
-      }
-      if (want_sym)
-        *reinterpret_cast<uint2*>(symc + uint64_t(tg + j) * 16) =
-            make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
-                       u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
     }
   }
   __syncthreads();
   if (nonfinite) set_status(p.status, CG_ERR_NONFINITE);
 
-  // ---- Phase C: histogram -> frequency table -> encoder constants.
+  // ---- Phase C: histograms -> frequency tables -> encoder constants (warp j
+  // normalises level j's table).
   if (want_hist) {
-    for (int u = tid; u < kAlphabet; u += kQThreads) {
+    for (int i = tid; i < NL * kAlphabet; i += kQThreads) {
+      const int j = i / kAlphabet, u = i - j * kAlphabet;
+      const uint32_t* hj = hist + j * kAlphabet * 32;
       uint32_t s = 0;
-      for (int j = 0; j < 32; ++j) s += hist[u * 32 + ((j + u) & 31)];
-      counts[u] = s;
+      for (int r = 0; r < 32; ++r) s += hj[u * 32 + ((r + u) & 31)];
+      counts[j * 256 + u] = s;
     }
     __syncthreads();
   }
-  if (warp == 0) {
+  if (warp < NL) {
+    const int j = warp;
     uint32_t f[8];
     if (mode == kModeSuppliedTables) {
       const uint16_t* fq = reinterpret_cast<const uint16_t*>(
@@ -452,12 +506,13 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
 #pragma unroll
       for (int i = 0; i < 8; ++i) f[i] = fq[lane * 8 + i];
     } else {
-      normalize_warp(counts, uint64_t(n) * D, f, lane);
+      normalize_warp(counts + j * 256, uint64_t(n) * D, f, lane);
     }
     uint32_t pk[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) pk[i] = f[2 * i] | (f[2 * i + 1] << 16);
     const uint4 fv = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    uint8_t* cont = cont_of(j);
     if (cont)
       reinterpret_cast<uint4*>(cont + sec.freq + uint64_t(tab) * 512)[lane] = fv;
     if (p.tables_out)
@@ -474,7 +529,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
         if (lane >= o) incl += v;
       }
       uint32_t cum = incl - local;
-      uint4* et = reinterpret_cast<uint4*>(p.etab) +
+      uint4* et = reinterpret_cast<uint4*>(NL == 1 ? p.etab : p.letab[j]) +
                   ((uint64_t(chunk) * L * 2 + slab) * H + h) * 256;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -676,7 +731,7 @@ __global__ void __launch_bounds__(kScanThreads) offsets_kernel(const EncParams p
     offs[n] = uint32_t(payload);  // == offsets[2 L n]
     cg_header hd;
     hd.magic = CG_MAGIC;
-    hd.version = CG_FORMAT_VERSION;
+    hd.version = p.adjacent ? CG_FORMAT_VERSION_ADJACENT : CG_FORMAT_VERSION;
     hd.level = uint8_t(p.level);
     hd.group = uint8_t(kGroup);
     hd.num_layers = uint32_t(L);
@@ -763,21 +818,13 @@ __global__ void __launch_bounds__(256) compact_kernel(const EncParams p) {
   }
 }
 
-}  // namespace
-
-cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stream) {
-  const int mode =
-      build_only ? kModeTablesOnly : (p.tables_in ? kModeSuppliedTables : kModeEncode);
-  const QSmem sm = q_smem();
-  cudaError_t err = cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(sm.total));
-  if (err != cudaSuccess) return err;
-  const uint64_t qblocks = uint64_t(p.num_chunks) * p.L * 2 * p.H;
-  quant_kernel<<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, mode);
-  if ((err = cudaGetLastError()) != cudaSuccess || build_only) return err;
+// rANS encode, offsets and compaction of one level's symbols (p.sym, p.etab,
+// p.slabtot) into its containers (p.out).
+cudaError_t launch_streams(const EncParams& p, bool check_f, cudaStream_t stream) {
+  cudaError_t err;
   const uint64_t tiles = (p.C + kRThreads - 1) / kRThreads;
   const unsigned rblocks = unsigned(uint64_t(p.num_chunks) * p.L * 2 * tiles);
-  if (mode == kModeSuppliedTables)
+  if (check_f)
     rans_kernel<true><<<rblocks, kRThreads, 0, stream>>>(p);
   else
     rans_kernel<false><<<rblocks, kRThreads, 0, stream>>>(p);
@@ -787,6 +834,47 @@ cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stre
   const uint64_t streams = uint64_t(p.num_chunks) * p.L * 2 * p.C;
   compact_kernel<<<unsigned((streams + 7) / 8), 256, 0, stream>>>(p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stream) {
+  const int mode =
+      build_only ? kModeTablesOnly : (p.tables_in ? kModeSuppliedTables : kModeEncode);
+  const QSmem sm = q_smem<1>();
+  auto* kern = p.adjacent ? quant_kernel<1, true> : quant_kernel<1, false>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm.total));
+  if (err != cudaSuccess) return err;
+  const uint64_t qblocks = uint64_t(p.num_chunks) * p.L * 2 * p.H;
+  kern<<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, mode);
+  if ((err = cudaGetLastError()) != cudaSuccess || build_only) return err;
+  return launch_streams(p, mode == kModeSuppliedTables, stream);
+}
+
+// Three levels from one quantiser pass: quant_kernel<3> writes every level's
+// symbols, tables and encoder constants; then each level's streams are encoded
+// and compacted in turn (the stream lengths and word slots are reused).
+cudaError_t launch_encode_levels(const EncParams& p, uint64_t* out_sizes, cudaStream_t stream) {
+  const QSmem sm = q_smem<3>();
+  cudaError_t err = cudaFuncSetAttribute(quant_kernel<3, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(sm.total));
+  if (err != cudaSuccess) return err;
+  const uint64_t qblocks = uint64_t(p.num_chunks) * p.L * 2 * p.H;
+  quant_kernel<3, false><<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, kModeEncode);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  for (int j = 0; j < 3; ++j) {
+    EncParams q = p;
+    q.level = j;
+    q.sym = p.lsym[j];
+    q.etab = p.letab[j];
+    q.slabtot = p.lslabtot[j];
+    q.out = p.lout[j];
+    q.out_sizes = out_sizes + uint64_t(j) * p.num_chunks;
+    if ((err = launch_streams(q, false, stream)) != cudaSuccess) return err;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace cg

@@ -56,23 +56,32 @@ class ChunkStore:
         return self.containers[(level, chunk)].numel()
 
 
-def encode_all_levels(kv: torch.Tensor, chunk_tokens: int, stream=None) -> ChunkStore:
+def encode_all_levels(kv: torch.Tensor, chunk_tokens: int, stream=None,
+                      chunks_per_call: int | None = None) -> ChunkStore:
     """Encode every chunk of kv ([L, 2, T, H, D], on the GPU) at the three
-    levels and keep the containers in pinned host memory (16-byte padded)."""
+    levels with cg_encode_levels (one read of the fp16 cache for all three)
+    and keep the containers in pinned host memory (16-byte padded).
+    chunks_per_call bounds the device workspace (default: all chunks)."""
     shape, T = ta._shape_of(kv)
     nch = -(-T // chunk_tokens)
+    per_call = min(nch, chunks_per_call or nch)
     store = ChunkStore(shape, chunk_tokens, nch)
-    enc = ta.Encoder(shape, chunk_tokens, nch, kv.device)
-    for level in LEVELS.values():
-        enc.encode(kv, level, stream=stream)
+    enc = ta.LevelsEncoder(shape, chunk_tokens, per_call, kv.device)
+    for k0 in range(0, nch, per_call):
+        m = min(per_call, nch - k0)
+        if m != enc.num_chunks:
+            enc = ta.LevelsEncoder(shape, chunk_tokens, m, kv.device)
+        views = enc.encode(kv, token_start=k0 * chunk_tokens, stream=stream)
         torch.cuda.synchronize(kv.device)
-        ta.raise_on_status(enc.status, "cg_encode")
-        sizes = enc.sizes.cpu().tolist()
-        for k in range(nch):
-            n = ((sizes[k] + 15) // 16) * 16
-            buf = torch.empty(n, dtype=torch.uint8, pin_memory=True)
-            buf.copy_(enc.out[k * enc.stride:k * enc.stride + n])
-            store.containers[(level, k)] = buf
+        ta.raise_on_status(enc.status, "cg_encode_levels")
+        for level in LEVELS.values():
+            sizes = views[level].sizes.cpu().tolist()
+            data = views[level].data
+            for k in range(m):
+                n = ((sizes[k] + 15) // 16) * 16
+                buf = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+                buf.copy_(data[k * enc.stride:k * enc.stride + n])
+                store.containers[(level, k0 + k)] = buf
     return store
 
 

@@ -8,12 +8,19 @@ other than the bench's, one JSON line per measurement.
 mistral7b  the Mistral-7B shape (one 1,536-token chunk) at the three levels;
 sweep      chunk sizes 512 / 1,024 / 1,536 / 2,048 x three levels x the two
            value distributions on the Mistral-7B shape at 32,768 tokens;
-llama34b   the Llama-34B shape (52 chunks) pre-encoded at the three levels,
-           then decoded chunk by chunk with cg_decode_into following the
+llama34b   the Llama-34B shape: first the three-level pre-encode of a
+           13-chunk batch, as three cg_encode calls and as one
+           cg_encode_levels call; then all 52 chunks pre-encoded at the three
+           levels and decoded chunk by chunk with cg_decode_into following the
            per-chunk level schedule: once from device-resident containers
            (kernel-only) and once streamed from pinned host memory with the
            next chunk's host-to-device copy overlapping the current decode
            (end to end).
+
+formats    format 1 (deltas to the group's anchor) against format 2 (deltas
+           between adjacent tokens): compression ratio and encode / decode
+           GB/s of both on the Llama-2-7B shape (balanced), the Mistral-7B
+           shape and the two sweep distributions at C = 1,536 (three levels).
 
 Every figure is fp16 bytes / device time (CUDA events on the launching
 stream, inputs resident unless stated, median of `--reps` after `--warmup`).
@@ -82,6 +89,70 @@ def run_grid(names, levels, chunk_sizes, dev, warmup, reps):
                 print(json.dumps(res), flush=True)
         del kv
         torch.cuda.empty_cache()
+
+
+def run_formats(dev, warmup, reps):
+    cells = [("llama2_7b", [1]), ("mistral7b", [0, 1, 2]), ("sweep_smooth", [0, 1, 2]),
+             ("sweep_rough", [0, 1, 2])]
+    stream = torch.cuda.current_stream(dev)
+    for name, levels in cells:
+        w = synth.WORKLOADS[name]
+        kv = _gen(w, dev)
+        shape = Shape(w.L, w.H, w.D)
+        C = 1536
+        nch = -(-w.T // C)
+        enc = ta.Encoder(shape, C, nch, dev)
+        out = torch.empty_like(kv)
+        status = ta.new_status(dev)
+        fp16 = kv.numel() * 2
+        for level in levels:
+            res = {"workload": name, "C": C, "level": level}
+            for fmt, adj in (("format1", False), ("format2", True)):
+                ms_e = _time(lambda: enc.encode(kv, level, stream=stream, adjacent=adj), stream,
+                             warmup, reps)
+                ms_d = _time(lambda: ta.decode_into(enc.out, enc.stride, shape, C, level, nch,
+                                                    out, status, stream=stream, adjacent=adj),
+                             stream, warmup, reps)
+                if ta.status_of(enc.status) != 0 or ta.status_of(status) != 0:
+                    raise RuntimeError(f"{name} {fmt}: status")
+                comp = int(enc.sizes.sum())
+                res[fmt] = {"ratio": round(fp16 / comp, 4), "encode_ms": round(ms_e, 3),
+                            "decode_ms": round(ms_d, 3),
+                            "encode_gbps": round(fp16 / ms_e / 1e6, 1),
+                            "decode_gbps": round(fp16 / ms_d / 1e6, 1)}
+            print(json.dumps(res), flush=True)
+        del kv, enc, out
+        torch.cuda.empty_cache()
+
+
+def run_preencode(dev, warmup, reps, batch=13):
+    """Three versions of a batch of chunks ([Practice] 2.1): three single-level
+    cg_encode calls against one cg_encode_levels call (one fp16 read)."""
+    w = synth.WORKLOADS["llama34b"]
+    kv = _gen(w, dev)
+    shape = Shape(w.L, w.H, w.D)
+    stream = torch.cuda.current_stream(dev)
+    single = ta.Encoder(shape, w.C, batch, dev)
+    ms_1 = _time(lambda: [single.encode(kv, lv, stream=stream) for lv in range(3)], stream,
+                 warmup, reps)
+    if ta.status_of(single.status) != 0:
+        raise RuntimeError("encode status")
+    del single
+    torch.cuda.empty_cache()
+    lev = ta.LevelsEncoder(shape, w.C, batch, dev)
+    ms_3 = _time(lambda: lev.encode(kv, stream=stream), stream, warmup, reps)
+    if ta.status_of(lev.status) != 0:
+        raise RuntimeError("encode_levels status")
+    fp16 = w.L * 2 * batch * w.C * w.H * w.D * 2
+    comp = [int(lev.sizes[j * batch:(j + 1) * batch].sum()) for j in range(3)]
+    print(json.dumps({"workload": "llama34b_preencode", "chunks": batch, "fp16_bytes": fp16,
+                      "ratio_per_level": [round(fp16 / c, 4) for c in comp],
+                      "three_encode_ms": round(ms_1, 3), "encode_levels_ms": round(ms_3, 3),
+                      "three_encode_gbps": round(fp16 / ms_1 / 1e6, 1),
+                      "encode_levels_gbps": round(fp16 / ms_3 / 1e6, 1),
+                      "speedup": round(ms_1 / ms_3, 3)}), flush=True)
+    del lev, kv
+    torch.cuda.empty_cache()
 
 
 def run_streamed(dev, warmup, reps):
@@ -170,7 +241,8 @@ def run_streamed(dev, warmup, reps):
 
 def main() -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("--config", choices=["mistral7b", "sweep", "llama34b"], required=True)
+    ap.add_argument("--config", choices=["mistral7b", "sweep", "llama34b", "formats"],
+                    required=True)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--reps", type=int, default=5)
     args = ap.parse_args()
@@ -182,7 +254,10 @@ def main() -> int:
         w = synth.WORKLOADS["sweep_smooth"]
         run_grid(["sweep_smooth", "sweep_rough"], [0, 1, 2], list(w.chunk_sizes), dev,
                  args.warmup, args.reps)
+    elif args.config == "formats":
+        run_formats(dev, args.warmup, args.reps)
     else:
+        run_preencode(dev, args.warmup, args.reps)
         run_streamed(dev, args.warmup, args.reps)
     return 0
 

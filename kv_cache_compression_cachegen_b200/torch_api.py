@@ -12,8 +12,10 @@ from dataclasses import dataclass
 
 import torch
 
-from . import (CG_OK, CacheGenError, Shape, cg_build_tables, cg_decode, cg_decode_into,
-               cg_decode_into_paged, cg_encode, cg_encode_workspace_bytes, cg_encoded_bound,
+from . import (CG_OK, CacheGenError, Shape, cg_build_tables, cg_decode, cg_decode_adjacent,
+               cg_decode_adjacent_into, cg_decode_into, cg_decode_into_paged, cg_encode,
+               cg_encode_adjacent, cg_encode_levels,
+               cg_encode_levels_workspace_bytes, cg_encode_workspace_bytes, cg_encoded_bound,
                cg_tables_bytes, check)
 
 
@@ -45,6 +47,7 @@ class Encoded:
     level: int
     shape: Shape
     status: torch.Tensor
+    adjacent: bool = False  # format 2 (deltas between adjacent tokens)
 
     def chunk(self, k: int) -> torch.Tensor:
         """Container k as a device view (synchronises to read its size)."""
@@ -66,23 +69,69 @@ class Encoder:
         self.status = new_status(device)
 
     def encode(self, kv: torch.Tensor, level: int, token_start: int = 0,
-               tables: torch.Tensor | None = None, stream=None) -> Encoded:
+               tables: torch.Tensor | None = None, stream=None,
+               adjacent: bool = False) -> Encoded:
+        """adjacent=True writes format 2 (cg_encode_adjacent; no supplied tables)."""
         shape, T = _shape_of(kv)
-        check(cg_encode(shape, kv, T, token_start, self.num_chunks, self.C, level, tables,
-                        self.out, self.stride, self.sizes, self.status, self.workspace,
-                        self.ws_bytes, stream), "cg_encode")
+        if adjacent:
+            if tables is not None:
+                raise ValueError("format 2 builds its own tables")
+            check(cg_encode_adjacent(shape, kv, T, token_start, self.num_chunks, self.C, level,
+                                     self.out, self.stride, self.sizes, self.status,
+                                     self.workspace, self.ws_bytes, stream),
+                  "cg_encode_adjacent")
+        else:
+            check(cg_encode(shape, kv, T, token_start, self.num_chunks, self.C, level, tables,
+                            self.out, self.stride, self.sizes, self.status, self.workspace,
+                            self.ws_bytes, stream), "cg_encode")
         return Encoded(self.out, self.sizes, self.stride, self.num_chunks, self.C, level, shape,
-                       self.status)
+                       self.status, adjacent)
+
+
+class LevelsEncoder:
+    """Workspace and output slots of cg_encode_levels for a fixed geometry:
+    the three levels' containers of num_chunks chunks, level-major."""
+
+    def __init__(self, shape: Shape, chunk_tokens: int, num_chunks: int, device,
+                 out_stride: int | None = None):
+        self.shape, self.C, self.num_chunks = shape, chunk_tokens, num_chunks
+        self.ws_bytes = cg_encode_levels_workspace_bytes(shape, chunk_tokens, num_chunks)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        self.stride = out_stride or cg_encoded_bound(shape, chunk_tokens)
+        self.out = torch.empty(3 * self.stride * num_chunks, dtype=torch.uint8, device=device)
+        self.sizes = torch.zeros(3 * num_chunks, dtype=torch.int64, device=device)
+        self.status = new_status(device)
+
+    def encode(self, kv: torch.Tensor, token_start: int = 0, stream=None) -> list[Encoded]:
+        """One Encoded view per level (HIGH, BALANCED, FAST)."""
+        shape, T = _shape_of(kv)
+        check(cg_encode_levels(shape, kv, T, token_start, self.num_chunks, self.C, self.out,
+                               self.stride, self.sizes, self.status, self.workspace,
+                               self.ws_bytes, stream), "cg_encode_levels")
+        per = self.stride * self.num_chunks
+        return [Encoded(self.out[j * per:(j + 1) * per],
+                        self.sizes[j * self.num_chunks:(j + 1) * self.num_chunks], self.stride,
+                        self.num_chunks, self.C, j, shape, self.status) for j in range(3)]
+
+
+def encode_levels(kv: torch.Tensor, chunk_tokens: int, token_start: int = 0,
+                  num_chunks: int | None = None, out_stride: int | None = None,
+                  stream=None) -> list[Encoded]:
+    shape, T = _shape_of(kv)
+    if num_chunks is None:
+        num_chunks = -(-(T - token_start) // chunk_tokens)
+    enc = LevelsEncoder(shape, chunk_tokens, num_chunks, kv.device, out_stride)
+    return enc.encode(kv, token_start, stream)
 
 
 def encode(kv: torch.Tensor, chunk_tokens: int, level: int, token_start: int = 0,
            num_chunks: int | None = None, tables: torch.Tensor | None = None,
-           out_stride: int | None = None, stream=None) -> Encoded:
+           out_stride: int | None = None, stream=None, adjacent: bool = False) -> Encoded:
     shape, T = _shape_of(kv)
     if num_chunks is None:
         num_chunks = -(-(T - token_start) // chunk_tokens)
     enc = Encoder(shape, chunk_tokens, num_chunks, kv.device, out_stride)
-    return enc.encode(kv, level, token_start, tables, stream)
+    return enc.encode(kv, level, token_start, tables, stream, adjacent)
 
 
 def build_tables(kv: torch.Tensor, chunk_tokens: int, level: int, token_start: int = 0,
@@ -100,27 +149,30 @@ def build_tables(kv: torch.Tensor, chunk_tokens: int, level: int, token_start: i
 
 def decode(data: torch.Tensor, stride: int, shape: Shape, chunk_tokens: int, level: int,
            num_chunks: int, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
-           stream=None):
-    """Decode into chunk slots [num_chunks][L][2][C][H][D] (chunk k packed by its n_k)."""
+           stream=None, adjacent: bool = False):
+    """Decode into chunk slots [num_chunks][L][2][C][H][D] (chunk k packed by its n_k).
+    adjacent=True decodes format-2 containers."""
     L, H, D = shape.num_layers, shape.num_kv_heads, shape.head_dim
     slot = L * 2 * chunk_tokens * H * D
     if out is None:
         out = torch.empty(slot * num_chunks, dtype=torch.int16, device=data.device)
     if status is None:
         status = new_status(data.device)
-    check(cg_decode(shape, data, stride, num_chunks, chunk_tokens, level, out, out.numel(),
-                    status, stream), "cg_decode")
+    fn = cg_decode_adjacent if adjacent else cg_decode
+    check(fn(shape, data, stride, num_chunks, chunk_tokens, level, out, out.numel(), status,
+             stream), fn.__name__)
     return out, status
 
 
 def decode_into(data: torch.Tensor, stride: int, shape: Shape, chunk_tokens: int, level: int,
                 num_chunks: int, kv: torch.Tensor, status: torch.Tensor | None = None,
-                stream=None):
+                stream=None, adjacent: bool = False):
     _, T = _shape_of(kv)
     if status is None:
         status = new_status(data.device)
-    check(cg_decode_into(shape, data, stride, num_chunks, chunk_tokens, level, kv, T, status,
-                         stream), "cg_decode_into")
+    fn = cg_decode_adjacent_into if adjacent else cg_decode_into
+    check(fn(shape, data, stride, num_chunks, chunk_tokens, level, kv, T, status, stream),
+          fn.__name__)
     return status
 
 

@@ -69,3 +69,48 @@ def test_argument_errors_are_synchronous(native_built):
     assert cg.cg_decode_into_paged(shp, 16, 64, 1, 256, 1, 16, 0, 16, 16, 64, 16,
                                    stream=0) == cg.CG_ERR_INVALID_ARG
     assert cg.cg_status_string(cg.CG_ERR_CORRUPT) == "corrupt container"
+
+
+def test_encode_levels_argument_checks(native_built):
+    import kv_cache_compression_cachegen_b200 as cg
+    shp = (4, 2, 64)
+    one = cg.cg_encode_workspace_bytes(shp, 256, 3)
+    three = cg.cg_encode_levels_workspace_bytes(shp, 256, 3)
+    # three symbol arrays and constant sets, one set of stream slots
+    assert one < three < 3 * one
+    bound = cg.cg_encoded_bound(shp, 256)
+    # missing pointers, no chunk, unaligned workspace: rejected before any launch
+    assert cg.cg_encode_levels(shp, None, 256, 0, 1, 256, 16, bound, 16, 16, 256, three,
+                               stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_encode_levels(shp, 16, 256, 0, 0, 256, 16, bound, 16, 16, 256, three,
+                               stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_encode_levels(shp, 16, 256, 0, 1, 256, 16, bound, 16, 16, 16, three,
+                               stream=0) == cg.CG_ERR_INVALID_ARG
+    # a workspace sized for one level, or an out stride without room for the tables
+    assert cg.cg_encode_levels(shp, 16, 256, 0, 1, 256, 16, bound, 16, 16, 256,
+                               cg.cg_encode_workspace_bytes(shp, 256, 1),
+                               stream=0) == cg.CG_ERR_CAPACITY
+    assert cg.cg_encode_levels(shp, 16, 256, 0, 1, 256, 16, 64, 16, 16, 256, three,
+                               stream=0) == cg.CG_ERR_CAPACITY
+
+
+def test_adjacent_format_argument_checks(native_built):
+    import kv_cache_compression_cachegen_b200 as cg
+    shp = (4, 2, 64)
+    ws = cg.cg_encode_workspace_bytes(shp, 256, 1)
+    bound = cg.cg_encoded_bound(shp, 256)
+    assert cg.cg_encode_adjacent(shp, None, 256, 0, 1, 256, 1, 16, bound, 16, 16, 256, ws,
+                                 stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_encode_adjacent(shp, 16, 256, 0, 1, 256, 3, 16, bound, 16, 16, 256, ws,
+                                 stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_encode_adjacent(shp, 16, 256, 0, 1, 256, 1, 16, bound, 16, 16, 256, ws - 256,
+                                 stream=0) == cg.CG_ERR_CAPACITY
+    assert cg.cg_decode_adjacent(shp, None, 64, 1, 256, 1, 16, 1 << 20, 16,
+                                 stream=0) == cg.CG_ERR_INVALID_ARG
+    assert cg.cg_decode_adjacent(shp, 16, 4096, 1, 256, 1, 16, 16, 16,
+                                 stream=0) == cg.CG_ERR_CAPACITY
+    assert cg.cg_decode_adjacent_into(shp, 16, 4096, 1, 256, 1, 16, 0, 16,
+                                      stream=0) == cg.CG_ERR_INVALID_ARG
+    # the two-pass grid of a huge call is refused up front
+    assert cg.cg_decode_adjacent((1024, 64, 256), 16, 4096, 100, 16384, 1, 16, 1 << 62, 16,
+                                 stream=0) in (cg.CG_ERR_UNSUPPORTED, cg.CG_ERR_CAPACITY)
