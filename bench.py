@@ -35,10 +35,10 @@ METRIC = "cg_decode / cg_encode GB/s (fp16 KV) on 1 B200, % of HBM roofline, com
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) per fp16 value of decode_kernel from one ncu capture
 # of the current kernel (profiles/decode_kernel_mistral7b_3072tok.md: 103.9 MB
-# read + 350.4 MB written for 32x2x3072x8x128 = 201,326,592 values); the bench
+# read + 352.8 MB written for 32x2x3072x8x128 = 201,326,592 values); the bench
 # reports it scaled by its own value count.  The capture ends with up to one L2
 # (126 MB) of written lines not yet in DRAM, so this slightly undercounts.
-DECODE_DRAM_BYTES_PER_VALUE = (103_941_888 + 350_364_160) / 201_326_592
+DECODE_DRAM_BYTES_PER_VALUE = (103_913_472 + 352_763_136) / 201_326_592
 
 
 def _peaks():
