@@ -147,7 +147,7 @@ typedef struct cg_shape {
 /* The 64-byte container header, exactly as stored. */
 typedef struct cg_header {
   uint32_t magic;         /* CG_MAGIC */
-  uint16_t version;       /* CG_FORMAT_VERSION */
+  uint16_t version;       /* CG_FORMAT_VERSION, or CG_FORMAT_VERSION_ADJACENT (format 2) */
   uint8_t level;          /* cg_level */
   uint8_t group;          /* CG_GROUP */
   uint32_t num_layers;    /* L */
