@@ -152,3 +152,40 @@ def test_formats_are_not_interchangeable():
     a = e1.data[:secs[2]].cpu().numpy()
     b = e2.data[:secs[2]].cpu().numpy()
     assert np.array_equal(a[secs[0]:], b[secs[0]:])
+
+
+def test_corrupt_format2_containers_report_a_status():
+    # both passes of the format-2 decode bound every read by the container and
+    # every write by the destination: damage comes back as a status
+    L, H, D, T, C = 3, 2, 32, 64, 32
+    kv = gu.gen(L, H, D, T, seed=21)
+    shape = Shape(L, H, D)
+    enc = ta.encode(kv, C, 1, adjacent=True)
+    torch.cuda.synchronize()
+    assert ta.status_of(enc.status) == 0
+    size0 = int(enc.sizes[0])
+    secs = oracle.sections(L, H, D, C)
+
+    def status(buf, stride, nch=2, into=False):
+        if into:
+            out = torch.zeros_like(kv)
+            st = ta.decode_into(buf, stride, shape, C, 1, nch, out, adjacent=True)
+        else:
+            _, st = ta.decode(buf, stride, shape, C, 1, nch, adjacent=True)
+        torch.cuda.synchronize()
+        return ta.status_of(st)
+
+    cut = (size0 // 16 - 1) * 16
+    assert status(enc.data[:cut].clone(), cut, nch=1) == oracle.CORRUPT
+    rng = np.random.default_rng(1)
+    for lo, hi in ((0, 64), (secs[2], secs[3]), (secs[3], secs[4]), (secs[4], size0)):
+        for _ in range(4):
+            buf = enc.data.clone()
+            buf[int(rng.integers(lo, hi))] ^= int(1 << rng.integers(0, 8))
+            for into in (False, True):
+                assert status(buf, enc.stride, into=into) in (0, oracle.CORRUPT,
+                                                              oracle.MISMATCH)
+    buf = enc.data.clone()
+    buf[secs[4] + 100] ^= 0x10
+    assert status(buf, enc.stride) == oracle.CORRUPT
+    assert status(torch.zeros_like(enc.data), enc.stride, into=True) == oracle.CORRUPT
