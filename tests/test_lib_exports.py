@@ -114,3 +114,18 @@ def test_adjacent_format_argument_checks(native_built):
     # the two-pass grid of a huge call is refused up front
     assert cg.cg_decode_adjacent((1024, 64, 256), 16, 4096, 100, 16384, 1, 16, 1 << 62, 16,
                                  stream=0) in (cg.CG_ERR_UNSUPPORTED, cg.CG_ERR_CAPACITY)
+
+
+def test_binding_signatures_match_the_header():
+    # every ctypes signature of the binding has as many arguments as the
+    # prototype declared in include/cachegen.h
+    import kv_cache_compression_cachegen_b200 as cg
+    text = re.sub(r"/\*.*?\*/", "", (ROOT / "include" / "cachegen.h").read_text(encoding="utf-8"),
+                  flags=re.S)
+    protos = {}
+    for m in re.finditer(r"\b(cg_[a-z_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        args = [a for a in m.group(2).split(",") if a.strip() and a.strip() != "void"]
+        protos[m.group(1)] = len(args)
+    assert set(cg._SIGNATURES) == set(protos), set(cg._SIGNATURES) ^ set(protos)
+    for name, (_, argtypes) in cg._SIGNATURES.items():
+        assert len(argtypes) == protos[name], (name, len(argtypes), protos[name])
