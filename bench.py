@@ -39,6 +39,25 @@ FALLBACK_HBM_GBS = 6650.0
 # reports it scaled by its own value count.  The capture ends with up to one L2
 # (126 MB) of written lines not yet in DRAM, so this slightly undercounts.
 DECODE_DRAM_BYTES_PER_VALUE = (103_913_472 + 352_763_136) / 201_326_592
+# Shared-memory wavefronts per warp-symbol of decode_kernel from the same
+# capture (48,259,107 wavefronts for 201,326,592 symbols): the random slot-table
+# lookups of 32 streams cost about four, the word refills, the reconstructed
+# anchors and the table fills the rest.  An SM serves one wavefront per clock.
+DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL = 48_259_107 / (201_326_592 / 32)
+
+
+def smem_ceiling(symbols: int, ms: float, sm_mhz, sms: int):
+    """The decode kernel against its shared-memory ceiling (one wavefront per
+    SM per clock at the SM clock sampled during the timed region)."""
+    if not sm_mhz or not ms or not sms:
+        return None
+    achieved = symbols / 32 * DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL / (ms * 1e-3)
+    peak = sms * float(sm_mhz) * 1e6
+    return {"bound": "smem", "achieved": round(achieved / 1e9, 1), "peak": round(peak / 1e9, 1),
+            "unit": "G wavefronts/s", "frac": round(achieved / peak, 4),
+            "wavefronts_per_warp_symbol": round(DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL, 2),
+            "source": "ncu wavefronts per warp-symbol of a 3,072-token Mistral-7B-shaped "
+                      "capture; peak = SMs x sampled SM clock"}
 
 
 def _peaks():
@@ -316,6 +335,10 @@ def run_ours(args):
             "gpu_launches": 5 * args.steps,
             "clocks": clocks,
         }
+        # what bounds the decode kernel instead of HBM: its shared-memory wavefronts
+        line["roofline"]["smem"] = smem_ceiling(
+            fp16_bytes // 2, ms_dec, clocks.get("sm_mhz"),
+            torch.cuda.get_device_properties(dev).multi_processor_count)
         if e2e is not None:
             line["e2e"] = e2e
         if not args.skip_cpu and world == 1:

@@ -61,3 +61,15 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
         steps, warmup, gpus = 1, 0, 2
 
     assert bench.run_reference(Args()) == 0
+
+
+def test_smem_ceiling_arithmetic():
+    # 32 x 10^9 symbols in 1 s at 7.67 wavefronts per warp-symbol on 148 SMs at
+    # 1965 MHz: 7.67e9 wavefronts/s against 290.8e9
+    got = bench.smem_ceiling(32_000_000_000, 1000.0, 1965.0, 148)
+    wf = bench.DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL
+    assert 7.6 < wf < 7.8
+    assert got["bound"] == "smem" and got["peak"] == round(148 * 1965e6 / 1e9, 1)
+    assert abs(got["achieved"] - wf) < 0.06
+    assert abs(got["frac"] - wf / 290.82) < 1e-3
+    assert bench.smem_ceiling(1, 1.0, None, 148) is None
