@@ -1,5 +1,7 @@
-// decode.cu -- fused rANS decode -> dequantise -> fp16 store (cg_decode and
-// cg_decode_into).
+// decode.cu -- fused rANS decode -> dequantise -> fp16 store (cg_decode,
+// cg_decode_into, cg_decode_into_paged), and the two-pass decode of format 2
+// (cg_decode_adjacent, cg_decode_adjacent_into: decode_kernel<true> stores the
+// symbols, chain_kernel rebuilds the adjacent-token chains; see chain_kernel).
 //
 // [Practice] 2.3 (parallel decode): the receiver decodes on the GPU with one
 // thread per token and hands the result to the thread that fills the model's
