@@ -17,6 +17,9 @@ llama34b   the Llama-34B shape: first the three-level pre-encode of a
            next chunk's host-to-device copy overlapping the current decode
            (end to end).
 
+paged      the Llama-2-7B shape (balanced) decoded into a paged pool of
+           16-token pages through a shuffled block table, against the flat
+           cg_decode_into of the same containers (and checked equal to it).
 formats    format 1 (deltas to the group's anchor) against format 2 (deltas
            between adjacent tokens): compression ratio and encode / decode
            GB/s of both on the Llama-2-7B shape (balanced), the Mistral-7B
@@ -89,6 +92,42 @@ def run_grid(names, levels, chunk_sizes, dev, warmup, reps):
                 print(json.dumps(res), flush=True)
         del kv
         torch.cuda.empty_cache()
+
+
+def run_paged(dev, warmup, reps, page_tokens=16):
+    w = synth.WORKLOADS["llama2_7b"]
+    kv = _gen(w, dev)
+    shape = Shape(w.L, w.H, w.D)
+    stream = torch.cuda.current_stream(dev)
+    nch, level = w.num_chunks, 1
+    enc = ta.encode(kv, w.C, level)
+    flat = torch.empty_like(kv)
+    status = ta.new_status(dev)
+    npages = -(-w.T // page_tokens)
+    table = torch.randperm(npages, generator=torch.Generator().manual_seed(0))
+    table = table.to(torch.int32).to(dev)
+    pool = torch.empty((w.L, 2, npages, page_tokens, w.H, w.D), dtype=torch.int16, device=dev)
+    ms_flat = _time(lambda: ta.decode_into(enc.data, enc.stride, shape, w.C, level, nch, flat,
+                                           status, stream=stream), stream, warmup, reps)
+    ms_paged = _time(lambda: ta.decode_into_paged(enc.data, enc.stride, shape, w.C, level, nch,
+                                                  pool, page_tokens, table, w.T, status,
+                                                  stream=stream), stream, warmup, reps)
+    if ta.status_of(enc.status) != 0 or ta.status_of(status) != 0:
+        raise RuntimeError("status")
+    # logical token t of the pool: row t % P of page table[t // P]
+    logical = pool[:, :, table.long()].reshape(w.L, 2, npages * page_tokens, w.H, w.D)
+    same = bool(torch.equal(logical[:, :, :w.T], flat))
+    fp16 = kv.numel() * 2
+    print(json.dumps({"workload": "llama2_7b_paged", "page_tokens": page_tokens,
+                      "pages": npages, "flat_decode_ms": round(ms_flat, 3),
+                      "paged_decode_ms": round(ms_paged, 3),
+                      "flat_decode_gbps": round(fp16 / ms_flat / 1e6, 1),
+                      "paged_decode_gbps": round(fp16 / ms_paged / 1e6, 1),
+                      "paged_equals_flat": same}), flush=True)
+    if not same:
+        raise RuntimeError("paged decode differs from the flat decode")
+    del kv, enc, flat, pool, logical
+    torch.cuda.empty_cache()
 
 
 def run_formats(dev, warmup, reps):
@@ -241,7 +280,7 @@ def run_streamed(dev, warmup, reps):
 
 def main() -> int:
     ap = argparse.ArgumentParser()
-    ap.add_argument("--config", choices=["mistral7b", "sweep", "llama34b", "formats"],
+    ap.add_argument("--config", choices=["mistral7b", "sweep", "llama34b", "formats", "paged"],
                     required=True)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--reps", type=int, default=5)
@@ -256,6 +295,8 @@ def main() -> int:
                  args.warmup, args.reps)
     elif args.config == "formats":
         run_formats(dev, args.warmup, args.reps)
+    elif args.config == "paged":
+        run_paged(dev, args.warmup, args.reps)
     else:
         run_preencode(dev, args.warmup, args.reps)
         run_streamed(dev, args.warmup, args.reps)

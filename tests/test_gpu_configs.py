@@ -54,6 +54,29 @@ def test_llama2_7b_full_size():
                            gu.chunk_slot(slots, shape, w.C, k, w.C))
 
 
+def test_llama2_7b_paged_pool_full_size():
+    """The bench workload decoded into a pool of 16-token pages through a shuffled
+    block table: every logical token's row equals the flat cg_decode_into."""
+    w = synth.WORKLOADS["llama2_7b"]
+    kv = gu.gen(w.L, w.H, w.D, w.T, w.seed, w.rho, w.p_out, w.m_out)
+    shape = Shape(w.L, w.H, w.D)
+    nch, P = w.num_chunks, 16
+    enc = ta.encode(kv, w.C, 1)
+    flat = torch.full_like(kv, 0x7E00)
+    st = ta.decode_into(enc.data, enc.stride, shape, w.C, 1, nch, flat)
+    npages = -(-w.T // P) + 3
+    table = torch.randperm(npages, generator=torch.Generator().manual_seed(5))
+    table = table[:-(-w.T // P)].to(torch.int32).cuda()
+    pool = torch.full((w.L, 2, npages, P, w.H, w.D), 0x7E00, dtype=torch.int16, device="cuda")
+    st2 = ta.decode_into_paged(enc.data, enc.stride, shape, w.C, 1, nch, pool, P, table, w.T)
+    torch.cuda.synchronize()
+    assert ta.status_of(enc.status) == 0 and ta.status_of(st) == 0 and ta.status_of(st2) == 0
+    logical = pool[:, :, table.long()].reshape(w.L, 2, table.numel() * P, w.H, w.D)
+    assert torch.equal(logical[:, :, :w.T], flat)
+    unused = sorted(set(range(npages)) - set(table.cpu().tolist()))
+    assert bool((pool[:, :, unused] == 0x7E00).all())
+
+
 def test_llama34b_streamed_decode_with_level_schedule():
     """Pre-encode every chunk at the three levels, keep the containers in pinned
     host memory, then decode chunk by chunk with cg_decode_into on one stream while
