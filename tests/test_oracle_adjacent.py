@@ -171,3 +171,36 @@ def test_container_format_2(oracle_lib):
     bad = c2.copy()
     bad[4] = 3  # no format 3
     assert oracle_lib.decode_chunk(bad, L, H, D, 20, 1, adjacent=True)[0] == oracle_lib.CORRUPT
+
+
+def test_format_2_streams_and_entropy_bound(oracle_lib):
+    # every stream of a format-2 container decodes to the format-2 symbols under
+    # tables built from those symbols, and the payload sits within 1 % (+ the
+    # per-stream flush) of the tables' information content, as in format 1
+    import struct
+    from kv_cache_compression_cachegen_b200 import synth
+    Lc, Hc, Dc, Tc = 4, 8, 128, 1536
+    kv = synth.generate_cpu(Lc, Hc, Dc, Tc, seed=1)
+    rc, cont = oracle_lib.encode_chunk(kv, 0, Tc, 1, adjacent=True)
+    assert rc == 0
+    rc, sym, _, _ = oracle_lib.quantize_chunk(kv, 0, Tc, 1, adjacent=True)
+    assert rc == 0
+    secs = oracle_lib.sections(Lc, Hc, Dc, Tc)
+    freq = np.frombuffer(cont[secs[2]:secs[3]].tobytes(), np.uint16).reshape(Lc, 2, Hc, 256)
+    assert np.array_equal(freq, oracle_lib.tables_of(sym))
+    payload = struct.unpack_from("<Q", bytes(cont[40:48]))[0]
+    offs = np.frombuffer(cont[secs[3]:secs[3] + 4 * (2 * Lc * Tc + 1)].tobytes(), np.uint32)
+    body = cont[secs[4]:secs[4] + payload]
+    for s in (0, 1, Tc - 1, Tc, 2 * Lc * Tc - 1):  # first, last and boundary streams
+        l, k, t = s // (2 * Tc), (s // Tc) % 2, s % Tc
+        words = np.frombuffer(body[offs[s]:offs[s + 1]].tobytes(), np.uint16)
+        rc, got = oracle_lib.rans_decode(words, Hc * Dc, Dc, freq[l, k])
+        assert rc == 0 and np.array_equal(got, sym[l, k, t].ravel())
+    f = np.take_along_axis(freq.astype(np.float64)[:, :, None, :, :].repeat(Tc, axis=2),
+                           sym.astype(np.int64).reshape(Lc, 2, Tc, Hc, Dc), axis=4)
+    info = float(np.sum(-np.log2(f / 4096.0)))
+    assert info <= 8 * payload <= 1.01 * info + 48 * 2 * Lc * Tc
+    # on this smooth AR(1) cache the adjacent differences carry less information
+    # than the differences to the anchor (the purpose of the format)
+    rc1, cont1 = oracle_lib.encode_chunk(kv, 0, Tc, 1)
+    assert rc1 == 0 and cont.size < cont1.size
