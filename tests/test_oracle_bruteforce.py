@@ -2,6 +2,11 @@
 KV cache: every code must be the argmin over all 255 codes of the reconstruction
 distance (equal distances away from zero), every zero point / scale must span the
 anchors' range, and every decoded value must be the fp16 of the reconstruction.
+Where the exact quotient lies so close to a half-integer that the float32
+quotient may round onto either side, the code must be the one the definition
+gives: roundf of the round-to-nearest float32 quotient (computed here in exact
+rationals), and every decoded value must be the two-rounding reconstruction
+RN(a + RN(q * s)) of the codes.
 """
 from fractions import Fraction
 
@@ -9,6 +14,13 @@ import numpy as np
 import pytest
 
 from exact import argmin_code, frac, near_half, rn_f32
+
+
+def _defn_code(d: Fraction, s: Fraction) -> int:
+    """clamp(roundf(RN(d / s))): the float32 quotient, halves away from zero."""
+    y = frac(rn_f32(d / s))
+    r = int(abs(y) + Fraction(1, 2))
+    return max(-127, min(127, r if y >= 0 else -r))
 
 L, H, D, T = 2, 1, 8, 20
 
@@ -31,6 +43,7 @@ def _expected_chunk(kv, t0, C, level, oracle_lib):
     zps = np.zeros((L, 2, H, D), dtype=np.float32)
     scs = np.zeros((L, 2, H, D), dtype=np.float32)
     fuzzy = np.zeros((L, 2, n, H, D), dtype=bool)
+    defn = np.zeros((L, 2, n, H, D), dtype=np.int64)
     for l in range(L):
         s = frac(oracle_lib.step(level, l, L))
         for kv_ in range(2):
@@ -44,11 +57,15 @@ def _expected_chunk(kv, t0, C, level, oracle_lib):
                 for g0 in range(0, n, 10):
                     xa = frac(col[g0])
                     if sc == 0:
-                        c = 0
+                        c = dfc = 0
                     else:
                         da = xa - frac(zp)
                         c = argmin_code(da, frac(sc))
                         fuzzy[l, kv_, g0, 0, d] = near_half(frac(rn_f32(da)), frac(sc))
+                        dfc = _defn_code(frac(rn_f32(da)), frac(sc))
+                        if fuzzy[l, kv_, g0, 0, d]:
+                            c = dfc  # the definition decides near a half
+                    defn[l, kv_, g0, 0, d] = dfc
                     ahat = rn_f32(frac(zp) + frac(rn_f32(c * frac(sc))))
                     sym[l, kv_, g0, 0, d] = c
                     dec[l, kv_, g0, 0, d] = ahat
@@ -56,9 +73,12 @@ def _expected_chunk(kv, t0, C, level, oracle_lib):
                         dd = frac(col[t]) - frac(ahat)
                         q = argmin_code(dd, s)
                         fuzzy[l, kv_, t, 0, d] = near_half(frac(rn_f32(dd)), s)
+                        defn[l, kv_, t, 0, d] = _defn_code(frac(rn_f32(dd)), s)
+                        if fuzzy[l, kv_, t, 0, d]:
+                            q = defn[l, kv_, t, 0, d]
                         sym[l, kv_, t, 0, d] = q
                         dec[l, kv_, t, 0, d] = rn_f32(frac(ahat) + frac(rn_f32(q * s)))
-    return sym, dec, zps, scs, fuzzy
+    return sym, dec, zps, scs, fuzzy, defn
 
 
 @pytest.mark.parametrize("C", [20, 16])
@@ -67,7 +87,7 @@ def _expected_chunk(kv, t0, C, level, oracle_lib):
 def test_bruteforce_tiny_cache(oracle_lib, C, level, seed):
     kv = _kv(seed)
     for t0 in range(0, T, C):
-        esym, edec, ezp, esc, fuzzy = _expected_chunk(kv, t0, C, level, oracle_lib)
+        esym, edec, ezp, esc, fuzzy, defn = _expected_chunk(kv, t0, C, level, oracle_lib)
         rc, sym, zp, sc = oracle_lib.quantize_chunk(kv, t0, C, level)
         assert rc == 0
         assert np.array_equal(zp.view(np.uint32), ezp.view(np.uint32))
@@ -76,13 +96,13 @@ def test_bruteforce_tiny_cache(oracle_lib, C, level, seed):
         exact = ~fuzzy
         assert np.array_equal(got[exact], esym[exact])
         assert np.all(np.abs(got[fuzzy] - esym[fuzzy]) <= 1)
+        assert np.array_equal(got, defn)  # the float32 quotient decides every code
         # the container round trip reproduces the reconstruction of these codes
         rc, cont = oracle_lib.encode_chunk(kv, t0, C, level)
         assert rc == 0
         rc, out, n, start = oracle_lib.decode_chunk(cont, L, H, D, C, level)
         assert rc == 0 and n == min(C, T - t0) and start == t0
-        if not fuzzy.any():
-            assert np.array_equal(out, edec.astype(np.float16).view(np.uint16))
+        assert np.array_equal(out, edec.astype(np.float16).view(np.uint16))
 
 
 def test_anchor_range_is_spanned(oracle_lib):
