@@ -93,9 +93,18 @@ def stream_decode(store: ChunkStore, levels: list[int], kv_out: torch.Tensor,
     dev = kv_out.device
     comp = stream or torch.cuda.current_stream(dev)
     copy = torch.cuda.Stream(dev)
-    status = status if status is not None else ta.new_status(dev)
+    own_status = status is None
+    status = ta.new_status(dev) if own_status else status
     maxb = max(store.size(levels[k], k) for k in range(store.num_chunks))
     stage = [torch.empty(maxb, dtype=torch.uint8, device=dev) for _ in range(2)]
+    # The buffers come from the current stream's pool but are written on `copy`
+    # and read on `comp`; tell the caching allocator, so that their memory is
+    # not handed out again before the work queued on those streams is done.
+    for buf in stage:
+        buf.record_stream(copy)
+        buf.record_stream(comp)
+    if own_status:
+        status.record_stream(comp)
     ready = [torch.cuda.Event() for _ in range(2)]
     done = [torch.cuda.Event() for _ in range(2)]
     for k in range(store.num_chunks):

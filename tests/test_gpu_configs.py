@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from kv_cache_compression_cachegen_b200 import Shape, synth
 from kv_cache_compression_cachegen_b200 import torch_api as ta
 
@@ -75,6 +76,12 @@ def test_llama2_7b_paged_pool_full_size():
     assert torch.equal(logical[:, :, :w.T], flat)
     unused = sorted(set(range(npages)) - set(table.cpu().tolist()))
     assert bool((pool[:, :, unused] == 0x7E00).all())
+    # sampled chunks of the pool's logical view against the oracle's decode
+    sampled = [0, 3, nch - 1]
+    dref = gu.oracle_decodes(gu.gpu_containers(enc, sampled), shape, w.C, 1)
+    for k in sampled:
+        got = gu.host(logical[:, :, k * w.C:(k + 1) * w.C])
+        assert np.array_equal(got, dref[k]), f"chunk {k} paged decode differs from the oracle"
 
 
 def test_llama34b_streamed_decode_with_level_schedule():
@@ -180,9 +187,47 @@ def test_bandwidth_adaptive_stream_decode():
         assert ta.status_of(st) == 0
         n = min(C, T - k * C)
         assert torch.equal(out[:, :, k * C:k * C + n], gu.chunk_slot(slot, shape, C, 0, n))
-    # the balanced versions also match the oracle
+    # every streamed chunk equals the oracle's decode of the container that was
+    # sent, and every sent container is the oracle's encoding of that chunk
     kv_h = gu.host(kv)
-    k = levels.index(1)
-    ref = gu.oracle_containers(kv_h, C, 1, [k])
-    got = store.containers[(1, k)].numpy()[:ref[k].size]
-    assert np.array_equal(got, ref[k])
+    got_all = gu.host(out)
+
+    def check(k):
+        lvl = levels[k]
+        rc, ref = oracle.encode_chunk(kv_h, k * C, C, lvl)
+        assert rc == 0
+        sent = store.containers[(lvl, k)].numpy()
+        assert np.array_equal(sent[:ref.size], ref) and not sent[ref.size:].any(), k
+        rc, vals, n, start = oracle.decode_chunk(ref, L, H, D, C, lvl)
+        assert rc == 0 and start == k * C
+        assert np.array_equal(got_all[:, :, k * C:k * C + n], vals), k
+    gu.pmap(check, list(range(store.num_chunks)))
+
+
+def test_stream_decode_on_a_side_stream():
+    """stream_decode given a stream other than the current one: its staging
+    buffers are released while the side stream still uses them, and the
+    current stream immediately allocates and overwrites memory; the decoded
+    cache must still equal the decode on the current stream."""
+    from kv_cache_compression_cachegen_b200 import streaming
+    L, H, D, C = 4, 2, 64, 256
+    T = 5 * C + 37
+    kv = gu.gen(L, H, D, T, seed=23)
+    store = streaming.encode_all_levels(kv, C)
+    levels = streaming.plan_levels([6.0, 2.0, 0.3, 7.0, 1.5])
+    ref = torch.full_like(kv, 0x7E00)
+    st = streaming.stream_decode(store, levels, ref)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == 0
+    side = torch.cuda.Stream()
+    out = torch.full_like(kv, 0x7E00)
+    torch.cuda.synchronize()
+    st2 = streaming.stream_decode(store, levels, out, stream=side)
+    # churn the current stream's allocator while the side stream works
+    junk = [torch.full((store.size(levels[k], k),), 0xAB, dtype=torch.uint8, device="cuda")
+            for k in range(store.num_chunks) for _ in range(4)]
+    del junk
+    side.synchronize()
+    torch.cuda.synchronize()
+    assert ta.status_of(st2) == 0
+    assert torch.equal(out, ref)

@@ -199,6 +199,13 @@ def test_decode_into_paged_pool():
     for lp in range(npages_logical):
         a, b = lp * P, min(T, (lp + 1) * P)
         assert torch.equal(pool[:, :, tab[lp], :b - a], flat[:, :, a:b]), lp
+    # every logical token's row also equals the oracle's decode of its chunk
+    conts = gu.gpu_containers(enc, range(nch))
+    dref = gu.oracle_decodes(conts, shape, C, 2)
+    logical = gu.host(pool[:, :, table.long()].reshape(L, 2, npages_logical * P, H, D))
+    for k in range(nch):
+        n = min(C, T - k * C)
+        assert np.array_equal(logical[:, :, k * C:k * C + n], dref[k]), k
     # pages no logical page maps to stay untouched
     unused = sorted(set(range(num_pages)) - set(tab))
     assert bool((pool[:, :, unused] == 0x7E00).all())
