@@ -330,7 +330,9 @@ cg_status cg_encode_levels(const cg_shape* shape, const uint16_t* kv_dev, int64_
  * every GPU that loads the library and held until the process exits; calls
  * whose cg_encode_workspace_bytes exceeds 128 MiB return CG_ERR_CAPACITY.  The
  * first call on a device looks up the block's device address (a host-side
- * query); make that first call before any stream capture.  Every call uses
+ * query), and so does the first call after the device's context was destroyed
+ * and created again (cudaDeviceReset); make that first call before any stream
+ * capture.  Every call uses
  * the same block, so calls that overlap on the GPU (other streams, other
  * host threads) race and must be serialised by the caller.  Nothing in the
  * block needs clearing: each call writes every byte it reads.  No allocation
