@@ -34,10 +34,10 @@ WORKLOAD = dict(name="llama2_7b", L=32, H=32, D=128, T=10752, C=1536, seed=2, rh
 METRIC = "cg_decode / cg_encode GB/s (fp16 KV) on 1 B200, % of HBM roofline, compression ratio"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) per fp16 value of decode_kernel from one ncu capture
-# of the current kernel (profiles/decode_kernel_mistral7b_3072tok.md: 103.9 MB
-# read + 352.8 MB written for 32x2x3072x8x128 = 201,326,592 values); the bench
-# reports it scaled by its own value count.  The capture ends with up to one L2
-# (126 MB) of written lines not yet in DRAM, so this slightly undercounts.
+# of the current kernel (103.9 MB read + 352.8 MB written for a Mistral-7B-shaped
+# 32x2x3072x8x128 case = 201,326,592 values); the bench reports it scaled by its
+# own value count.  The capture ends with up to one L2 (126 MB) of written lines
+# not yet in DRAM, so this slightly undercounts.
 DECODE_DRAM_BYTES_PER_VALUE = (103_913_472 + 352_763_136) / 201_326_592
 # Shared-memory wavefronts per warp-symbol of decode_kernel from the same
 # capture (48,259,107 wavefronts for 201,326,592 symbols): the random slot-table
@@ -149,11 +149,19 @@ def job_gbps(bytes_per_rank, world, ms):
     return bytes_per_rank * world / ms / 1e6
 
 
+def host_cores() -> int:
+    """Cores this process may run on (the affinity mask, else the CPU count)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
 def _oracle_sample(threads: int):
     """The CPU sample: one chunk of the workload cut into 16 independent 2-head
     slices ([32, 2, 1536, 2, 128] each, 50 MB of fp16), round-tripped through the
-    oracle on up to `threads` host threads."""
-    import numpy as np
+    oracle as max(16, threads) tasks (the slices in turn) on `threads` host
+    threads, so that every core has work."""
     import oracle
     from concurrent.futures import ThreadPoolExecutor
     from kv_cache_compression_cachegen_b200 import synth
@@ -162,6 +170,7 @@ def _oracle_sample(threads: int):
     slices = [synth.generate_cpu(w["L"], 2, w["D"], w["C"], seed=w["seed"] * 100 + i,
                                  rho=w["rho"], p_out=w["p_out"], m_out=w["m_out"])
               for i in range(16)]
+    tasks = [slices[i % len(slices)] for i in range(max(16, threads))]
 
     def run_one(kv):
         rc, cont = oracle.encode_chunk(kv, 0, w["C"], w["level"])
@@ -170,14 +179,15 @@ def _oracle_sample(threads: int):
         assert rc == 0
         return cont.size
 
-    nbytes = sum(s.nbytes for s in slices)
-    desc = (f"one {w['C']}-token chunk of the {w['name']} workload as 16 slices of "
-            f"[{w['L']},2,{w['C']},2,{w['D']}] fp16 ({nbytes / 1e6:.0f} MB), encode+decode")
+    nbytes = sum(s.nbytes for s in tasks)
+    desc = (f"{len(tasks)} tasks over 16 slices of [{w['L']},2,{w['C']},2,{w['D']}] fp16 "
+            f"(one {w['C']}-token chunk of the {w['name']} workload cut by head pairs), "
+            f"{nbytes / 1e6:.0f} MB encode+decode")
 
     def step():
         t0 = time.perf_counter()
         with ThreadPoolExecutor(threads) as ex:
-            sizes = list(ex.map(run_one, slices))
+            sizes = list(ex.map(run_one, tasks))
         return time.perf_counter() - t0, sizes
 
     def one_core():
@@ -194,7 +204,7 @@ def run_reference(args):
     rank, world, _ = _env_rank()
     if rank != 0:
         return 0
-    threads = max(1, min(16, os.cpu_count() or 1))
+    threads = host_cores()
     step, nbytes, desc = _oracle_sample(threads)
     for _ in range(args.warmup):
         step()
@@ -225,6 +235,7 @@ def run_ours(args):
     import kv_cache_compression_cachegen_b200 as cg
     from kv_cache_compression_cachegen_b200 import synth
     from kv_cache_compression_cachegen_b200 import torch_api as ta
+    from kv_cache_compression_cachegen_b200.stats import clamp_counts
 
     rank, world, local = _env_rank()
     if world > 1:
@@ -246,13 +257,19 @@ def run_ours(args):
     status = ta.new_status(dev)
     fp16_bytes = kv.numel() * 2
 
+    nvtx = torch.cuda.nvtx
+
     def encode():
+        nvtx.range_push("cg_encode")
         cg.check(cg.cg_encode(shape, kv, T, 0, nch, C, level, None, enc.out, enc.stride,
                               enc.sizes, enc.status, enc.workspace, enc.ws_bytes, stream))
+        nvtx.range_pop()
 
     def decode():
+        nvtx.range_push("cg_decode_into")
         cg.check(cg.cg_decode_into(shape, enc.out, enc.stride, nch, C, level, kv_out, T, status,
                                    stream))
+        nvtx.range_pop()
 
     torch.cuda.synchronize(dev)
     for _ in range(max(args.warmup, 0)):
@@ -294,12 +311,23 @@ def run_ours(args):
     alg = fp16_bytes + comp_bytes
     enc_frac = alg / ms_enc / 1e6 / hbm
     dec_frac = alg / ms_dec / 1e6 / hbm
+    # the target's own roofline definition: the same bytes over 8 TB/s
+    enc_frac_8 = alg / ms_enc / 1e6 / 8000.0
+    dec_frac_8 = alg / ms_dec / 1e6 / 8000.0
+    clamped, deltas = clamp_counts(kv, kv_out, C, level)
 
     # ---- end to end through the C ABI with host buffers --------------------
     e2e = None
     if not args.skip_e2e:
         e2e = _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, C,
                    level, T, fp16_bytes, world, dist)
+        full = _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, C,
+                    level, T, fp16_bytes, world, dist, kv_back=True)
+        e2e["with_decoded_kv_to_host"] = {
+            "value": full["value"], "unit": full["unit"], "ms_per_step": full["ms_per_step"],
+            "d2h_bytes_per_step": full["d2h_bytes_per_step"],
+            "note": "the same step with every decoded chunk also copied back to pinned host "
+                    "memory"}
 
     line = None
     if rank == 0:
@@ -319,11 +347,16 @@ def run_ours(args):
                        "parallelism": f"dp{world} (independent caches per GPU)"},
             "encode_gbps": round(enc_gbps, 2), "decode_gbps": round(dec_gbps, 2),
             "encode_ms": round(ms_enc, 4), "decode_ms": round(ms_dec, 4),
-            "encode_roofline_frac": round(enc_frac, 4), "decode_roofline_frac": round(dec_frac, 4),
-            "decode_frac_of_8tbs": round(alg / ms_dec / 1e6 / 8000.0, 4),
-            "encode_frac_of_8tbs": round(alg / ms_enc / 1e6 / 8000.0, 4),
+            "encode_roofline_frac": round(enc_frac_8, 4),
+            "decode_roofline_frac": round(dec_frac_8, 4),
+            "roofline_frac_definition": "(fp16 bytes + container bytes) / 8 TB/s / time",
+            "encode_frac_of_measured_hbm": round(enc_frac, 4),
+            "decode_frac_of_measured_hbm": round(dec_frac, 4),
             "compression_ratio": round(fp16_bytes / comp_bytes, 4),
             "container_bytes": comp_bytes,
+            "clamp_rate": clamped / deltas,
+            "clamp_rate_def": "delta values whose code hit the [-127, 127] clamp (reconstruction "
+                              "error above step/2 + half an fp16 spacing), over all delta values",
             "roofline": {"kernel": "decode_kernel (cg_decode_into)", "bound": "hbm",
                          "achieved": round(alg / ms_dec / 1e6, 1), "peak": hbm,
                          "peak_source": f"{peak_src} hbm_gbs", "unit": "GB/s",
@@ -352,23 +385,26 @@ def run_ours(args):
 
 
 def _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, C, level, T,
-         fp16_bytes, world, dist):
+         fp16_bytes, world, dist, kv_back=False):
     """Host in, host out, chunk by chunk: pinned fp16 KV -> H2D -> cg_encode ->
     D2H container (the sender's side), then H2D container -> cg_decode_into ->
     D2H status (the receiver's side; the decoded KV stays in device memory, where
     the model reads it).  Three streams overlap the copies of one chunk with the
     compute of another: `h2d` carries the fp16 chunks, `d2h` the containers out,
-    `back` the containers in; `stream` runs the kernels."""
+    `back` the containers in; `stream` runs the kernels.  kv_back=True also
+    copies every decoded chunk back to pinned host memory (on `d2h`)."""
     L = shape.num_layers
     host_kv = torch.empty(kv.shape, dtype=kv.dtype, pin_memory=True)
     host_kv.copy_(kv)
+    host_out = torch.empty(kv.shape, dtype=kv.dtype, pin_memory=True) if kv_back else None
     host_cont = torch.empty(enc.out.numel(), dtype=torch.uint8, pin_memory=True)
     host_status = torch.empty(2, dtype=torch.int32, pin_memory=True)
     sizes = enc.sizes.cpu().tolist()
     dev_cont = torch.empty_like(enc.out)
     h2d, d2h, back = (torch.cuda.Stream(dev) for _ in range(3))
     ev = lambda: torch.cuda.Event()  # noqa: E731
-    kv_in, enc_done, out_done, in_done = ([ev() for _ in range(nch)] for _ in range(4))
+    kv_in, enc_done, out_done, in_done, dec_done = ([ev() for _ in range(nch)]
+                                                    for _ in range(5))
     torch.cuda.synchronize(dev)
     steps = max(1, min(args.steps, 3))
     t0 = torch.cuda.Event(enable_timing=True)
@@ -405,6 +441,14 @@ def _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, 
             stream.wait_event(in_done[k])
             cg.check(cg.cg_decode_into(shape, dev_cont[o:], enc.stride, 1, C, level, kv_out, T,
                                        status, stream))
+            if kv_back:
+                dec_done[k].record(stream)
+                a, b = k * C, min(T, (k + 1) * C)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(dec_done[k])
+                    for l in range(L):
+                        for kvi in range(2):
+                            host_out[l, kvi, a:b].copy_(kv_out[l, kvi, a:b], non_blocking=True)
         with torch.cuda.stream(stream):
             host_status[0:1].copy_(status, non_blocking=True)
             host_status[1:2].copy_(enc.status, non_blocking=True)
@@ -414,15 +458,18 @@ def _e2e(args, torch, cg, ta, shape, kv, enc, kv_out, status, stream, dev, nch, 
     torch.cuda.synchronize(dev)
     if int(host_status[0]) != 0 or int(host_status[1]) != 0:
         raise RuntimeError(f"e2e status {host_status.tolist()}")
+    if kv_back and not torch.equal(host_out[:, :, :C], kv_out[:, :, :C].cpu()):
+        raise RuntimeError("e2e: decoded KV copied back differs from the device copy")
     ms = reduce_max([t0.elapsed_time(t1) / steps], world, dist, dev)[0]
     comp = sum(sizes)
     return {"value": round(job_gbps(fp16_bytes, world, ms), 3), "unit": "GB/s",
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": fp16_bytes + comp,
-            "d2h_bytes_per_step": comp + 8, "overlap": "per-chunk copies on three streams"}
+            "d2h_bytes_per_step": comp + 8 + (fp16_bytes if kv_back else 0),
+            "overlap": "per-chunk copies on three streams"}
 
 
 def _cpu_baseline():
-    threads = max(1, min(16, os.cpu_count() or 1))
+    threads = host_cores()
     step, nbytes, desc = _oracle_sample(threads)
     dt, _ = step()
     dt1, nb1 = step.one_core()

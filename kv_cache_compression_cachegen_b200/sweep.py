@@ -27,7 +27,8 @@ formats    format 1 (deltas to the group's anchor) against format 2 (deltas
 
 Every figure is fp16 bytes / device time (CUDA events on the launching
 stream, inputs resident unless stated, median of `--reps` after `--warmup`).
-Status words are checked after every run.
+Status words are checked after every run.  clamp_rate is the share of delta
+values whose code hit the [-127, 127] clamp (stats.clamp_counts).
 """
 from __future__ import annotations
 
@@ -40,6 +41,7 @@ import torch
 from . import Shape, library
 from . import synth
 from . import torch_api as ta
+from .stats import clamp_counts
 
 
 def _time(fn, stream, warmup: int, reps: int) -> float:
@@ -68,9 +70,11 @@ def _cell(kv, shape, T, C, level, stream, warmup, reps):
         raise RuntimeError(f"status {ta.status_of(enc.status)} / {ta.status_of(status)}")
     fp16 = kv.numel() * 2
     comp = int(enc.sizes.sum())
+    clamped, deltas = clamp_counts(kv, out, C, level)
     return {"C": C, "level": level, "chunks": nch, "encode_ms": round(ms_e, 4),
             "decode_ms": round(ms_d, 4), "encode_gbps": round(fp16 / ms_e / 1e6, 1),
-            "decode_gbps": round(fp16 / ms_d / 1e6, 1), "ratio": round(fp16 / comp, 4)}
+            "decode_gbps": round(fp16 / ms_d / 1e6, 1), "ratio": round(fp16 / comp, 4),
+            "clamp_rate": clamped / deltas}
 
 
 def _gen(w, dev):
