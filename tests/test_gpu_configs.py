@@ -214,7 +214,8 @@ def test_stream_decode_on_a_side_stream():
     T = 5 * C + 37
     kv = gu.gen(L, H, D, T, seed=23)
     store = streaming.encode_all_levels(kv, C)
-    levels = streaming.plan_levels([6.0, 2.0, 0.3, 7.0, 1.5])
+    levels = streaming.plan_levels([6.0, 2.0, 0.3, 7.0, 1.5, 0.8])
+    assert len(levels) == store.num_chunks
     ref = torch.full_like(kv, 0x7E00)
     st = streaming.stream_decode(store, levels, ref)
     torch.cuda.synchronize()
