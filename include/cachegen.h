@@ -276,17 +276,16 @@ cg_status cg_encode_adjacent(const cg_shape* shape, const uint16_t* kv_dev, int6
                              uint64_t* out_sizes_dev, int32_t* status_dev, void* workspace_dev,
                              uint64_t workspace_bytes, cudaStream_t stream);
 
-/* cg_decode of format-2 containers (same arguments and layout).  Two launches:
- * the rANS pass leaves every value's symbol (u16) in its destination slot,
- * then a second kernel rebuilds each group's chain in place.  As in every
- * decode call, a slot whose chunk or stream is reported corrupt holds
- * undefined values. */
+/* cg_decode of format-2 containers (same arguments and layout).  The decoder
+ * rebuilds each group's chain from its anchor in the same pass that decodes
+ * the streams.  As in every decode call, a slot whose chunk or stream is
+ * reported corrupt holds undefined values. */
 cg_status cg_decode_adjacent(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
                              int32_t num_chunks, int32_t chunk_tokens, cg_level level,
                              uint16_t* out_dev, uint64_t out_elems, int32_t* status_dev,
                              cudaStream_t stream);
 
-/* cg_decode_into of format-2 containers (same arguments, same two passes). */
+/* cg_decode_into of format-2 containers (same arguments). */
 cg_status cg_decode_adjacent_into(const cg_shape* shape, const uint8_t* in_dev,
                                   uint64_t in_stride, int32_t num_chunks, int32_t chunk_tokens,
                                   cg_level level, uint16_t* kv_dev, int64_t total_tokens,

@@ -340,17 +340,6 @@ cg_status cg_decode_into(const cg_shape* shape, const uint8_t* in_dev, uint64_t 
                        1, total_tokens, status_dev, stream);
 }
 
-// Format 2 decodes in two launches: the rANS pass leaves the symbols in the
-// destination, then chain_kernel rebuilds the values (one CTA of 256 threads
-// per 256 (group, 8-channel block) pairs of a (chunk, layer, K/V)).
-static cg_status check_chain_grid(const cg_shape* shape, int32_t num_chunks,
-                                  int32_t chunk_tokens) {
-  const uint64_t work = uint64_t((chunk_tokens + CG_GROUP - 1) / CG_GROUP) *
-                        (uint64_t(shape->num_kv_heads) * shape->head_dim / 8);
-  const uint64_t blocks = uint64_t(num_chunks) * shape->num_layers * 2 * ((work + 255) / 256);
-  return blocks > 0x7FFFFFFFull ? CG_ERR_UNSUPPORTED : CG_OK;
-}
-
 cg_status cg_decode_adjacent(const cg_shape* shape, const uint8_t* in_dev, uint64_t in_stride,
                              int32_t num_chunks, int32_t chunk_tokens, cg_level level,
                              uint16_t* out_dev, uint64_t out_elems, int32_t* status_dev,
@@ -358,7 +347,6 @@ cg_status cg_decode_adjacent(const cg_shape* shape, const uint8_t* in_dev, uint6
   cg_status st = check_decode_args(shape, in_dev, in_stride, num_chunks, chunk_tokens, level,
                                    out_dev, status_dev);
   if (st != CG_OK) return st;
-  if ((st = check_chain_grid(shape, num_chunks, chunk_tokens)) != CG_OK) return st;
   const uint64_t slot = uint64_t(shape->num_layers) * 2 * chunk_tokens * shape->num_kv_heads *
                         shape->head_dim;
   if (out_elems < slot * uint64_t(num_chunks)) return CG_ERR_CAPACITY;
@@ -373,7 +361,6 @@ cg_status cg_decode_adjacent_into(const cg_shape* shape, const uint8_t* in_dev,
   cg_status st = check_decode_args(shape, in_dev, in_stride, num_chunks, chunk_tokens, level,
                                    kv_dev, status_dev);
   if (st != CG_OK) return st;
-  if ((st = check_chain_grid(shape, num_chunks, chunk_tokens)) != CG_OK) return st;
   if (total_tokens < 1) return CG_ERR_INVALID_ARG;
   const uint64_t elems = uint64_t(shape->num_layers) * 2 * uint64_t(total_tokens) *
                          shape->num_kv_heads * shape->head_dim;

@@ -172,7 +172,7 @@ struct DecParams {
   int num_chunks;
   int C, L, H, D;
   int level;
-  int adjacent;            // 1: format 2 containers; decode writes codes, then rebuilds chains
+  int adjacent;            // 1: format 2 containers (each delta against the previous token)
   uint16_t* out;
   uint64_t out_elems;      // size of out in elements (checked against the shape by the C ABI)
   int into;                // 0: chunk slots [L][2][n][H][D]; 1: full KV [L][2][T][H][D];

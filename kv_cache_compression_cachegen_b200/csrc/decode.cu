@@ -1,26 +1,35 @@
-// decode.cu -- fused rANS decode -> dequantise -> fp16 store (cg_decode,
-// cg_decode_into, cg_decode_into_paged), and the two-pass decode of format 2
-// (cg_decode_adjacent, cg_decode_adjacent_into: decode_kernel<true> stores the
-// symbols, chain_kernel rebuilds the adjacent-token chains; see chain_kernel).
+// decode.cu -- fused rANS decode -> dequantise -> fp16 store: cg_decode,
+// cg_decode_into, cg_decode_into_paged, and the format-2 calls
+// cg_decode_adjacent / cg_decode_adjacent_into.
 //
 // [Practice] 2.3 (parallel decode): the receiver decodes on the GPU with one
 // thread per token and hands the result to the thread that fills the model's
 // KV cache.  Here one thread owns one rANS stream, i.e. one (layer, K/V,
-// token), and writes its fp16 values straight into the destination layout, so
-// decode and fill are one kernel.
+// token), and the same kernel writes the fp16 values into the destination
+// layout, so decode and fill are one kernel.
 //
-// CTA = one "unit": 32 anchor groups (320 tokens) of one (chunk, layer, K/V).
-//   warp 0      decodes the 32 anchor streams (lane g -> token 10 g);
-//   warps 1..9  decode the 288 delta streams (9 per group).
+// CTA = one "unit": 32 anchor groups (320 tokens) of one (chunk, layer, K/V);
+// thread t decodes the stream of local token t (anchors and deltas alike).
 // Every stream holds H*D symbols in [h][d] order and every head has its own
-// frequency table, so the CTA walks the heads in lockstep:
-//   iteration it:  anchor warp decodes head it      with table it % 3,
-//                  delta warps decode head it - 1   with table (it-1) % 3,
-//                  all threads fill the slot table of head it + 1,
-//                  one warp scans the frequencies of head it + 2.
-// The anchor warp runs one head ahead so that the reconstructed anchors a_g of
-// head it-1 (fp32, in shared memory) are ready when the delta warps need them;
-// one __syncthreads per head separates the iterations.
+// frequency table, so the CTA walks the heads in lockstep, two phases per head:
+//
+//   phase A  every thread decodes the D symbols of head h of its stream and
+//            leaves the byte codes u = q + 127 in shared memory, codes[t][d];
+//            the only shared-memory traffic is the slot-table lookup, the word
+//            refill and one 8-byte code store per 8 symbols.
+//   phase B  the threads turn the codes of head h into fp16.  A work item is
+//            (anchor group g, channel pair): the anchor value
+//            a = zp + (float)c * scale, then the nine deltas a + (float)q * step
+//            (format 2: each delta against the previous token's value), all
+//            fp32 with IEEE round-to-nearest adds and multiplies (no
+//            contraction), stored as fp16 pairs; the 32 lanes of a warp take
+//            32 consecutive pairs of one token row, so every store instruction
+//            writes whole 32-byte sectors.  Meanwhile the slot table of head
+//            h + 1 is built and the zero points / scales of head h + 1 staged.
+//
+// A __syncthreads separates the phases.  Anchors get no special treatment in
+// phase A, and the reconstructed anchors never leave the registers of the
+// phase-B item, so the work of a head is spread evenly over the CTA.
 //
 // Compressed words reach a thread through a 64-byte ring in shared memory
 // (four 16-byte blocks, plus a copy of the first block after the last, so that
@@ -29,18 +38,6 @@
 // issued two steps earlier; since 8 symbols consume at most 8 words (one
 // block), the words a step can read were always requested at least two steps
 // before, so global-memory latency stays off the decode chain.
-//
-// Per symbol: one slot-table lookup, the state update, an optional 16-bit
-// refill from the ring, and the dequantisation a + (float)q * s with IEEE
-// round-to-nearest adds and multiplies (no contraction).  The slot entry keeps
-// the symbol in its top byte, so (float)q comes from a byte permute and one
-// exact subtraction instead of a second shared-memory lookup.
-//
-// Output: a thread's values of two steps (16 fp16, 32 contiguous bytes of its
-// token's row) leave as one 256-bit store, a full L2 sector.  Every thread
-// writes its own row, so a warp's store touches 32 rows; with 16-byte stores
-// the L2 had to take twice as many partial-sector writes, which bounded the
-// kernel more than the decoding itself.
 #include <cuda_fp16.h>
 
 #include "cg_common.cuh"
@@ -49,10 +46,9 @@ namespace cg {
 namespace {
 
 constexpr int kUnitGroups = 32;
-constexpr int kDeltaPerGroup = kGroup - 1;             // 9
-constexpr int kWarps = 1 + kDeltaPerGroup;             // anchor warp + 9 delta warps
-constexpr int kThreads = 32 * kWarps;                  // 320
-constexpr int kUnitTokens = kUnitGroups * kGroup;      // 320
+constexpr int kThreads = kUnitGroups * kGroup;         // 320: one stream per thread
+constexpr int kWarps = kThreads / 32;                  // 10
+constexpr int kUnitTokens = kThreads;
 constexpr uint32_t kCumBuf = 800;                      // bytes per compacted-table buffer
 constexpr uint32_t kRingBytes = 64;                    // per thread: 4 blocks of 16 bytes
 constexpr uint32_t kRingBlocks = kRingBytes / 16;
@@ -61,26 +57,32 @@ constexpr uint32_t kRingStride = kRingBytes + 16;       // + a copy of slot 0 af
 
 // Dynamic shared memory layout (byte offsets), a function of H and D.
 struct DecSmem {
-  uint32_t tbl;     // u32 [3][4096]  slot tables, packed (u << 24) | (f << 12) | (slot - cum)
-  uint32_t ahat;    // f32 [2][32][D + 4]  reconstructed anchors of the last two heads
+  uint32_t tbl;     // u32 [2][4096]  slot tables, packed (u << 24) | (f << 12) | (slot - cum)
+  uint32_t codes;   // u8  [320][D + 8]  symbols u of the current head, one row per token
   uint32_t ring;    // u8  [320][80]  per-thread word rings: 4 slots + a mirror of slot 0
-  uint32_t cum;     // [2] x {u16 pcum[257], u8 psym[256], i32 nz}: the next two heads' present
-                    //        symbols in order and their cumulative frequencies
-  uint32_t zs;      // f32 [2][2][D]  zero points and scales of the anchor warp's next heads
+  uint32_t cum;     // [2] x {u16 pcum[257], u8 psym[256], i32 nz}: compacted tables of
+                    //        the next heads (present symbols in order, cumulative freqs)
+  uint32_t zs;      // f32 [2][2][D]  zero points and scales of the current and next head
+  uint32_t rows;    // u64 [320]      destination row of each token (0: not written)
+  uint32_t ok;      // u8  [320]      1 when the token's stream is being decoded
   uint32_t single;  // i32 [H]        symbol of a one-symbol table, else -1
   uint32_t total;
 };
 
 __host__ __device__ inline uint32_t al16(uint32_t v) { return (v + 15u) & ~15u; }
 
+__host__ __device__ inline uint32_t codes_stride(int D) { return uint32_t(D) + 8u; }
+
 __host__ __device__ inline DecSmem dec_smem(int H, int D) {
   DecSmem s;
   s.tbl = 0;
-  s.ahat = al16(s.tbl + 3u * 4096u * 4u);
-  s.ring = al16(s.ahat + 2u * kUnitGroups * uint32_t(D + 4) * 4u);
+  s.codes = s.tbl + 2u * 4096u * 4u;
+  s.ring = al16(s.codes + uint32_t(kThreads) * codes_stride(D));
   s.cum = al16(s.ring + uint32_t(kThreads) * kRingStride);
   s.zs = al16(s.cum + 2u * kCumBuf);
-  s.single = al16(s.zs + 4u * uint32_t(D) * 4u);
+  s.rows = al16(s.zs + 4u * uint32_t(D) * 4u);
+  s.ok = al16(s.rows + uint32_t(kThreads) * 8u);
+  s.single = al16(s.ok + uint32_t(kThreads));
   s.total = al16(s.single + uint32_t(H) * 4u);
   return s;
 }
@@ -253,10 +255,15 @@ __device__ __forceinline__ uint32_t ring_rebase(uint32_t ra, uint32_t rb) {
   return rb + ((ra - rb) & (kRingBytes - 1));
 }
 
-// (float)(u - 127) for the symbol u in the entry's top byte: the bits
-// 0x4B0000uu are the float 2^23 + u, and subtracting 2^23 + 127 is exact.
-__device__ __forceinline__ float sym_value(uint32_t e) {
-  return __fsub_rn(__uint_as_float(__byte_perm(e, 0x4B000000u, 0x7653)), 8388735.0f);
+// The symbols u (top bytes of four slot entries) as four bytes of one word.
+__device__ __forceinline__ uint32_t pack4(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t e3) {
+  return __byte_perm(__byte_perm(e0, e1, 0x0073), __byte_perm(e2, e3, 0x0073), 0x5410);
+}
+
+// (float)(u - 127) for a symbol byte u: the bits 0x4B0000uu are the float
+// 2^23 + u, and subtracting 2^23 + 127 is exact.
+__device__ __forceinline__ float code_value(uint32_t u) {
+  return __fsub_rn(__uint_as_float(0x4B000000u | u), 8388735.0f);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -264,122 +271,8 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Stream position of a thread: p (absolute word index of the next unread
-// word, kept per step) and ra (its ring address, advanced per refill).
-struct Pos {
-  uint32_t p, ra, w;
-};
-
-// 32-byte store of 16 fp16 values (one full sector); two 16-byte stores when
-// the destination is only 16-byte aligned.
-__device__ __forceinline__ void store16h(uint16_t* dst, const uint32_t (&hv)[8], bool al32) {
-  if (al32) {
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"l"(dst),
-                 "r"(hv[0]), "r"(hv[1]), "r"(hv[2]), "r"(hv[3]), "r"(hv[4]), "r"(hv[5]),
-                 "r"(hv[6]), "r"(hv[7])
-                 : "memory");
-  } else {
-    *reinterpret_cast<uint4*>(dst) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    *reinterpret_cast<uint4*>(dst + 8) = make_uint4(hv[4], hv[5], hv[6], hv[7]);
-  }
-}
-
-// The symbol u = q + 127 of a packed slot entry (format 2's first pass stores
-// the symbols themselves, as u16, in the destination).
-__device__ __forceinline__ uint32_t pack_codes(uint32_t e0, uint32_t e1) {
-  return (e0 >> 24) | ((e1 >> 8) & 0x00FF0000u);
-}
-
-// Delta lane: decode head h of its stream in steps of 8 values; the values of
-// two steps leave as one 32-byte store.  CODES: the symbols instead of values.
-template <bool CODES>
-__device__ __forceinline__ void decode_delta_head(uint32_t& x, Pos& ps, Ring& r,
-                                                  const uint32_t* __restrict__ tbl, float step,
-                                                  const float* __restrict__ arow,
-                                                  uint16_t* __restrict__ orow, int D, bool al32) {
-  for (int d0 = 0; d0 < D; d0 += 16) {
-    uint32_t hv[8];
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int dd = d0 + 8 * half;
-      ring_issue(r, ps.p);
-      ring_wait_two_steps();
-      ps.ra = ring_rebase(ps.ra, r.rb);
-      const uint32_t ra0 = ps.ra;
-      const float4 a0 = *reinterpret_cast<const float4*>(arow + dd);
-      const float4 a1 = *reinterpret_cast<const float4*>(arow + dd + 4);
-      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-      for (int k = 0; k < 8; k += 2) {
-        const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl);
-        const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl);
-        if constexpr (CODES) {
-          hv[4 * half + (k >> 1)] = pack_codes(e0, e1);
-        } else {
-          const float v0 = __fadd_rn(a[k], __fmul_rn(sym_value(e0), step));
-          const float v1 = __fadd_rn(a[k + 1], __fmul_rn(sym_value(e1), step));
-          hv[4 * half + (k >> 1)] = pack_half2(v0, v1);
-        }
-      }
-      ps.p += (ps.ra - ra0) >> 1;
-    }
-    store16h(orow + d0, hv, al32);
-  }
-}
-
-// Anchor lane: decode head h, write fp16(a) and keep a (fp32) for the deltas.
-// zp and sc point at the head's zero points and scales staged in shared memory.
-// CODES: store the symbols only (format 2 rebuilds the values afterwards).
-template <bool CODES>
-__device__ __forceinline__ void decode_anchor_head(uint32_t& x, Pos& ps, Ring& r,
-                                                   const uint32_t* __restrict__ tbl,
-                                                   const float* __restrict__ zp,
-                                                   const float* __restrict__ sc,
-                                                   float* __restrict__ arow,
-                                                   uint16_t* __restrict__ orow, int D, bool al32) {
-  for (int d0 = 0; d0 < D; d0 += 16) {
-    uint32_t hv[8];
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int dd = d0 + 8 * half;
-      ring_issue(r, ps.p);
-      ring_wait_two_steps();
-      ps.ra = ring_rebase(ps.ra, r.rb);
-      const uint32_t ra0 = ps.ra;
-      const float4 z0 = *reinterpret_cast<const float4*>(zp + dd);
-      const float4 z1 = *reinterpret_cast<const float4*>(zp + dd + 4);
-      const float4 s0 = *reinterpret_cast<const float4*>(sc + dd);
-      const float4 s1 = *reinterpret_cast<const float4*>(sc + dd + 4);
-      const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-      const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-      if constexpr (CODES) {
-#pragma unroll
-        for (int k = 0; k < 8; k += 2) {
-          const uint32_t e0 = rans_step(x, ps.ra, ps.w, tbl);
-          const uint32_t e1 = rans_step(x, ps.ra, ps.w, tbl);
-          hv[4 * half + (k >> 1)] = pack_codes(e0, e1);
-        }
-        ps.p += (ps.ra - ra0) >> 1;
-      } else {
-        float v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t e = rans_step(x, ps.ra, ps.w, tbl);
-          v[k] = __fadd_rn(z[k], __fmul_rn(sym_value(e), s[k]));
-        }
-        ps.p += (ps.ra - ra0) >> 1;
-        *reinterpret_cast<float4*>(arow + dd) = make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4*>(arow + dd + 4) = make_float4(v[4], v[5], v[6], v[7]);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) hv[4 * half + k] = pack_half2(v[2 * k], v[2 * k + 1]);
-      }
-    }
-    store16h(orow + d0, hv, al32);
-  }
-}
-
-// Header validation of one container (both decode kernels run it; every CTA
-// of a chunk checks the same 64 bytes).  Returns 0 or the status to report.
+// Header validation of one container (every CTA of a chunk checks the same
+// 64 bytes).  Returns 0 or the status to report.
 __device__ int check_header(const uint8_t* base, const DecParams& p, cg_header& h) {
   const uint4* hp = reinterpret_cast<const uint4*>(base);
   uint4* hd = reinterpret_cast<uint4*>(&h);
@@ -427,7 +320,77 @@ __device__ __forceinline__ uint16_t* dest_row(const DecParams& p, int chunk, int
          ((uint64_t(slab) * n + t) * H) * D;
 }
 
-template <bool CODES>
+// Phase A for one head: decode D symbols of the thread's stream with the slot
+// table tb and leave their codes in the thread's row of the code buffer.
+__device__ __forceinline__ void decode_codes(uint32_t& x, uint32_t& p, uint32_t& ra,
+                                             uint32_t& w, Ring& r,
+                                             const uint32_t* __restrict__ tb,
+                                             uint8_t* __restrict__ crow, int D) {
+  for (int d0 = 0; d0 < D; d0 += 8) {
+    ring_issue(r, p);
+    ring_wait_two_steps();
+    ra = ring_rebase(ra, r.rb);
+    const uint32_t ra0 = ra;
+    const uint32_t e0 = rans_step(x, ra, w, tb);
+    const uint32_t e1 = rans_step(x, ra, w, tb);
+    const uint32_t e2 = rans_step(x, ra, w, tb);
+    const uint32_t e3 = rans_step(x, ra, w, tb);
+    const uint32_t e4 = rans_step(x, ra, w, tb);
+    const uint32_t e5 = rans_step(x, ra, w, tb);
+    const uint32_t e6 = rans_step(x, ra, w, tb);
+    const uint32_t e7 = rans_step(x, ra, w, tb);
+    p += (ra - ra0) >> 1;
+    *reinterpret_cast<uint2*>(crow + d0) = make_uint2(pack4(e0, e1, e2, e3), pack4(e4, e5, e6, e7));
+  }
+}
+
+// Phase B for one head: fp16 values from the codes.  Item (group g, channel
+// pair j): the anchor's pair, then the pair of each later token of the group.
+// A warp takes 32 consecutive pairs of one group (a "segment"), so each store
+// instruction writes 128 contiguous bytes of one token row; the segments are
+// dealt to the warps in turn.
+template <bool ADJ>
+__device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, uint32_t cstride,
+                                             const float* __restrict__ zh,
+                                             const uint64_t* __restrict__ rows,
+                                             const uint8_t* __restrict__ ok, int ngroups,
+                                             int ntok, int h, int D, float step, int warp,
+                                             int lane) {
+  const int P = D >> 1;                 // channel pairs per token row
+  const int S = (P + 31) >> 5;          // segments of 32 pairs per row
+  for (int wi = warp; wi < ngroups * S; wi += kWarps) {
+    const int g = S == 3 ? wi / 3 : wi >> (S >> 1);  // S is 1, 2, 3 or 4 (D <= 256)
+    const int j = (wi - g * S) * 32 + lane;
+    const int t0 = g * kGroup;
+    if (j >= P || !ok[t0]) continue;  // past the row, or the anchor was rejected: untouched
+    const float2 z = *reinterpret_cast<const float2*>(zh + 2 * j);
+    const float2 sc = *reinterpret_cast<const float2*>(zh + D + 2 * j);
+    const uint32_t c = *reinterpret_cast<const uint16_t*>(codes + t0 * cstride + 2 * j);
+    float a0 = __fadd_rn(z.x, __fmul_rn(code_value(c & 0xFFu), sc.x));
+    float a1 = __fadd_rn(z.y, __fmul_rn(code_value(c >> 8), sc.y));
+    const uint32_t col = uint32_t(h * D + 2 * j);
+    uint16_t* r0 = reinterpret_cast<uint16_t*>(rows[t0]);
+    if (r0) *reinterpret_cast<uint32_t*>(r0 + col) = pack_half2(a0, a1);
+    const int tend = min(t0 + kGroup, ntok);
+    for (int t = t0 + 1; t < tend; ++t) {
+      if (!ok[t]) {
+        if (ADJ) break;  // the chain has lost a link: the rest of the group stays untouched
+        continue;
+      }
+      const uint32_t q = *reinterpret_cast<const uint16_t*>(codes + t * cstride + 2 * j);
+      const float v0 = __fadd_rn(a0, __fmul_rn(code_value(q & 0xFFu), step));
+      const float v1 = __fadd_rn(a1, __fmul_rn(code_value(q >> 8), step));
+      uint16_t* rt = reinterpret_cast<uint16_t*>(rows[t]);
+      if (rt) *reinterpret_cast<uint32_t*>(rt + col) = pack_half2(v0, v1);
+      if (ADJ) {  // format 2: the next token's delta is taken against this value
+        a0 = v0;
+        a1 = v1;
+      }
+    }
+  }
+}
+
+template <bool ADJ>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_ok, s_n, s_bad;
@@ -459,13 +422,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   const int n = s_n;
   const int unit_t0 = unit * kUnitTokens;
   if (unit_t0 >= n) return;
+  const int ntok = min(kUnitTokens, n - unit_t0);   // tokens of this unit
+  const int ngroups = (ntok + kGroup - 1) / kGroup;
 
   const Sections sec = sections(L, H, D, n);
   const DecSmem sm = dec_smem(H, D);
   uint32_t* tbl = reinterpret_cast<uint32_t*>(smem + sm.tbl);
-  float* ahat = reinterpret_cast<float*>(smem + sm.ahat);
+  uint8_t* codes = smem + sm.codes;
+  const uint32_t cstride = codes_stride(D);
+  uint64_t* rows = reinterpret_cast<uint64_t*>(smem + sm.rows);
+  uint8_t* okf = smem + sm.ok;
   int* single = reinterpret_cast<int*>(smem + sm.single);
-  const int astride = D + 4;
+  float* zs = reinterpret_cast<float*>(smem + sm.zs);  // [2][{zp, scale}][D]
   const int warp = tid >> 5, lane = tid & 31;
   const int slab = l * 2 + kv;
 
@@ -493,8 +461,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
     }
   }
   const float step = step_of(p.level, l, L);
-  // 32-byte stores need a 32-byte aligned destination (rows are multiples of 32 bytes)
-  const bool al32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
   __syncthreads();
   if (s_bad) {
     if (tid == 0) set_status(p.status, CG_ERR_CORRUPT);
@@ -504,40 +470,30 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   if (warp < 2 && warp < H)
     cum_compact(__ldg(reinterpret_cast<const uint4*>(freq + warp * 256) + lane),
                 cum_buf(cumb + warp * kCumBuf), lane);
+  const float* zp_sec = reinterpret_cast<const float*>(base + sec.zp) + size_t(slab) * H * D;
+  const float* sc_sec = reinterpret_cast<const float*>(base + sec.scale) + size_t(slab) * H * D;
+  for (int i = tid; i < 2 * D; i += kThreads)
+    zs[i] = i < D ? __ldg(zp_sec + i) : __ldg(sc_sec + (i - D));
   __syncthreads();
   fill_table(tbl, cum_buf(cumb), tid);
 
-  // This thread's stream.
-  int g_local, token;
-  if (warp == 0) {
-    g_local = lane;
-    token = unit_t0 + kGroup * lane;
-  } else {
-    const int k = (warp - 1) * 32 + lane;
-    g_local = k / kDeltaPerGroup;
-    token = unit_t0 + kGroup * g_local + 1 + k % kDeltaPerGroup;
-  }
-  bool active = token < n;
-  const uint32_t* offs = reinterpret_cast<const uint32_t*>(base + sec.offsets);
-  // Destination row of this thread's token (a paged pool's block table may
-  // leave it unmapped: nothing is written for it).
-  uint16_t* orow = p.out;
+  // This thread's stream: local token unit_t0 + tid.
+  const int token = unit_t0 + tid;
+  bool active = tid < ntok;
+  uint64_t orow = 0;
   if (active) {
-    orow = dest_row(p, chunk, slab, n, s_tstart, token);
-    if (orow == nullptr) {
-      set_status(p.status, CG_ERR_MISMATCH);
-      active = false;
-      orow = p.out;
-    }
+    uint16_t* r = dest_row(p, chunk, slab, n, s_tstart, token);
+    if (r == nullptr) set_status(p.status, CG_ERR_MISMATCH);  // unmapped page: not written
+    orow = reinterpret_cast<uint64_t>(r);
   }
+  const uint32_t* offs = reinterpret_cast<const uint32_t*>(base + sec.offsets);
   Ring ring;
   ring.gbase = base;
   const uint32_t rings = uint32_t(__cvta_generic_to_shared(smem + sm.ring));
   ring.rb = rings + uint32_t(tid) * kRingStride;
   ring.lim = uint32_t(s_total / 16);
   ring.fb = 0;
-  Pos ps{0u, ring.rb, 0u};
-  uint32_t pend = 0, x = kRansL;
+  uint32_t x = kRansL, pw = 0, pend = 0, ra = ring.rb, w = 0;
   if (active) {
     const uint64_t s = uint64_t(slab) * n + token;
     const uint32_t o0 = __ldg(offs + s), o1 = __ldg(offs + s + 1);
@@ -546,177 +502,70 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
       set_status(p.status, CG_ERR_CORRUPT);
       active = false;
     } else {
-      uint32_t pw = uint32_t((sec.payload + o0) / 2);
+      pw = uint32_t((sec.payload + o0) / 2);
       pend = uint32_t((sec.payload + o1) / 2);
       ring.fb = pw >> 3;
       for (uint32_t i = 0; i < kRingBlocks; ++i) ring_issue(ring, pw);
       ring_wait_all();
       x = (lds_u16(ring_addr(ring, pw)) << 16) | lds_u16(ring_addr(ring, pw + 1));
       pw += 2;
-      ps.p = pw;
-      ps.ra = ring_addr(ring, pw);
-      ps.w = lds_u16(ps.ra);
+      ra = ring_addr(ring, pw);
+      w = lds_u16(ra);
       if (x < kRansL) {
         set_status(p.status, CG_ERR_CORRUPT);
         active = false;
       }
     }
   }
-  const float* zp_sec = reinterpret_cast<const float*>(base + sec.zp) + size_t(slab) * H * D;
-  const float* sc_sec = reinterpret_cast<const float*>(base + sec.scale) + size_t(slab) * H * D;
-  float* zs = reinterpret_cast<float*>(smem + sm.zs);  // [2][{zp, scale}][D]
-  for (int i = tid; i < 2 * D; i += kThreads)
-    zs[i] = i < D ? __ldg(zp_sec + i) : __ldg(sc_sec + (i - D));
+  rows[tid] = orow;
+  okf[tid] = active ? 1 : 0;
+  uint8_t* crow = codes + tid * cstride;
   __syncthreads();
 
-  for (int it = 0; it <= H; ++it) {
-    // Global loads for the next heads are issued first and consumed after this
-    // iteration's decode, so their latency never delays the barrier.
-    const bool scan_warp = it + 2 < H && warp == it % kWarps;
+  for (int h = 0; h < H; ++h) {
+    // ---- phase A: the codes of head h
+    if (active) {
+      const int one = single[h];
+      if (one >= 0) {  // a one-symbol table: the state stays put, no word is read
+        const uint32_t cc = uint32_t(one) * 0x01010101u;
+        for (int d0 = 0; d0 < D; d0 += 8) *reinterpret_cast<uint2*>(crow + d0) = make_uint2(cc, cc);
+      } else {
+        decode_codes(x, pw, ra, w, ring, tbl + (h & 1) * kM, crow, D);
+      }
+    }
+    // global loads for the next heads are issued before the barrier
+    const bool scan_warp = h + 2 < H && warp == h % kWarps;
     uint4 fq = make_uint4(0, 0, 0, 0);
-    if (scan_warp) fq = __ldg(reinterpret_cast<const uint4*>(freq + (it + 2) * 256) + lane);
+    if (scan_warp) fq = __ldg(reinterpret_cast<const uint4*>(freq + (h + 2) * 256) + lane);
     float zv[2] = {0.0f, 0.0f};
-    const bool stage = it + 1 < H;
+    const bool stage = h + 1 < H;
     if (stage) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int i = tid + j * kThreads;
         if (i < 2 * D)
-          zv[j] = i < D ? __ldg(zp_sec + (it + 1) * D + i) : __ldg(sc_sec + (it + 1) * D + (i - D));
-      }
-      fill_table(tbl + ((it + 1) % 3) * kM, cum_buf(cumb + ((it + 1) & 1) * kCumBuf), tid);
-    }
-    if (warp == 0) {
-      if (it < H && active) {
-        const int h = it;
-        const uint32_t* tb = tbl + (h % 3) * kM;
-        float* arow = ahat + ((h & 1) * kUnitGroups + g_local) * astride;
-        const float* zh = zs + (h & 1) * 2 * D;
-        const int one = single[h];
-        if (one >= 0 && CODES) {
-          const uint32_t cc = uint32_t(one) * 0x10001u;
-          for (int d0 = 0; d0 < D; d0 += 8)
-            *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(cc, cc, cc, cc);
-        } else if (one >= 0) {
-          const float c = float(one - 127);
-          for (int d0 = 0; d0 < D; d0 += 8) {
-            float v[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = __fadd_rn(zh[d0 + k], __fmul_rn(c, zh[D + d0 + k]));
-#pragma unroll
-            for (int k = 0; k < 8; ++k) arow[d0 + k] = v[k];
-            *reinterpret_cast<uint4*>(orow + h * D + d0) =
-                make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]),
-                           pack_half2(v[4], v[5]), pack_half2(v[6], v[7]));
-          }
-        } else {
-          decode_anchor_head<CODES>(x, ps, ring, tb, zh, zh + D, arow, orow + h * D, D, al32);
-        }
-      }
-    } else if (it >= 1 && active) {
-      const int h = it - 1;
-      const uint32_t* tb = tbl + (h % 3) * kM;
-      const float* arow = ahat + ((h & 1) * kUnitGroups + g_local) * astride;
-      const int one = single[h];
-      if (one >= 0 && CODES) {
-        const uint32_t cc = uint32_t(one) * 0x10001u;
-        for (int d0 = 0; d0 < D; d0 += 8)
-          *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(cc, cc, cc, cc);
-      } else if (one >= 0) {
-        const float v = __fmul_rn(float(one - 127), step);
-        for (int d0 = 0; d0 < D; d0 += 8) {
-          uint32_t hv[4];
-#pragma unroll
-          for (int k = 0; k < 8; k += 2)
-            hv[k >> 1] = pack_half2(__fadd_rn(arow[d0 + k], v), __fadd_rn(arow[d0 + k + 1], v));
-          *reinterpret_cast<uint4*>(orow + h * D + d0) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        }
-      } else {
-        decode_delta_head<CODES>(x, ps, ring, tb, step, arow, orow + h * D, D, al32);
+          zv[j] = i < D ? __ldg(zp_sec + (h + 1) * D + i) : __ldg(sc_sec + (h + 1) * D + (i - D));
       }
     }
-    if (scan_warp) cum_compact(fq, cum_buf(cumb + (it & 1) * kCumBuf), lane);
+    __syncthreads();
+    // ---- phase B: fp16 values of head h; the table, zero points and scales
+    // of head h + 1, the compacted table of head h + 2
+    dequant_head<ADJ>(codes, cstride, zs + (h & 1) * 2 * D, rows, okf, ngroups, ntok, h, D, step,
+                      warp, lane);
     if (stage) {
-      float* zn = zs + ((it + 1) & 1) * 2 * D;
+      fill_table(tbl + ((h + 1) & 1) * kM, cum_buf(cumb + ((h + 1) & 1) * kCumBuf), tid);
+      float* zn = zs + ((h + 1) & 1) * 2 * D;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int i = tid + j * kThreads;
         if (i < 2 * D) zn[i] = zv[j];
       }
     }
+    if (scan_warp) cum_compact(fq, cum_buf(cumb + (h & 1) * kCumBuf), lane);
     __syncthreads();
   }
   ring_wait_all();
-  if (active && (x != kRansL || ps.p != pend)) set_status(p.status, CG_ERR_CORRUPT);
-}
-
-// ---- format 2, second pass -------------------------------------------------
-// decode_kernel<true> has left every value's symbol u = q + 127 (a u16) in its
-// destination slot.  One thread per (anchor group, 8 channels of the token
-// row) rebuilds the group's chain in place: the anchor a = zp + c * scale,
-// then x^_t = x^_(t-1) + q_t * step for the group's later tokens, each sum and
-// product rounded to nearest (no contraction), each value stored as fp16.  The
-// ten rows' symbols are loaded before the first store, so a thread keeps ten
-// 16-byte loads in flight; a warp covers 512 contiguous bytes of each row.
-constexpr int kChainThreads = 256;
-
-__global__ void __launch_bounds__(kChainThreads) chain_kernel(const DecParams p,
-                                                              const int blocks_per_slab) {
-  __shared__ int s_ok, s_n;
-  __shared__ long long s_tstart;
-  const int tid = threadIdx.x;
-  const int part = blockIdx.x % blocks_per_slab;
-  const int rest = blockIdx.x / blocks_per_slab;
-  const int slab = rest % (2 * p.L);
-  const int chunk = rest / (2 * p.L);
-  const int L = p.L, H = p.H, D = p.D;
-  const uint8_t* base = p.in + uint64_t(chunk) * p.in_stride;
-  if (tid == 0) {
-    cg_header h;
-    s_ok = check_header(base, p, h) == 0;  // the decode pass has reported any error
-    s_n = int(h.n_tokens);
-    s_tstart = (long long)h.token_start;
-  }
-  __syncthreads();
-  if (!s_ok) return;
-  const int n = s_n;
-  const int rb = H * D / 8;  // 8-channel blocks of a token row
-  const int64_t w = int64_t(part) * kChainThreads + tid;
-  if (w >= int64_t((n + kGroup - 1) / kGroup) * rb) return;
-  const int g = int(w / rb), c0 = int(w % rb) * 8;
-  const int t0 = g * kGroup, ntok = min(kGroup, n - t0);
-  const Sections sec = sections(L, H, D, n);
-  const float* zp = reinterpret_cast<const float*>(base + sec.zp) + uint64_t(slab) * H * D + c0;
-  const float* sc = reinterpret_cast<const float*>(base + sec.scale) + uint64_t(slab) * H * D + c0;
-  const float4 z0 = __ldg(reinterpret_cast<const float4*>(zp));
-  const float4 z1 = __ldg(reinterpret_cast<const float4*>(zp + 4));
-  const float4 s0 = __ldg(reinterpret_cast<const float4*>(sc));
-  const float4 s1 = __ldg(reinterpret_cast<const float4*>(sc + 4));
-  const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-  const float sa[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-  const float step = step_of(p.level, slab >> 1, L);
-
-  uint16_t* rows[kGroup];
-  uint4 cv[kGroup];
-#pragma unroll
-  for (int r = 0; r < kGroup; ++r) {
-    rows[r] = r < ntok ? dest_row(p, chunk, slab, n, s_tstart, t0 + r) : nullptr;
-    cv[r] = rows[r] ? *reinterpret_cast<const uint4*>(rows[r] + c0) : make_uint4(0, 0, 0, 0);
-  }
-  float x[8];
-#pragma unroll
-  for (int r = 0; r < kGroup; ++r) {
-    if (rows[r] == nullptr) break;  // end of the chunk (or an unmapped page)
-    const uint32_t cw[4] = {cv[r].x, cv[r].y, cv[r].z, cv[r].w};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float q = float(int((cw[k >> 1] >> (16 * (k & 1))) & 0xFFFFu) - 127);
-      x[k] = r == 0 ? __fadd_rn(z[k], __fmul_rn(q, sa[k])) : __fadd_rn(x[k], __fmul_rn(q, step));
-    }
-    *reinterpret_cast<uint4*>(rows[r] + c0) =
-        make_uint4(pack_half2(x[0], x[1]), pack_half2(x[2], x[3]), pack_half2(x[4], x[5]),
-                   pack_half2(x[6], x[7]));
-  }
+  if (active && (x != kRansL || pw != pend)) set_status(p.status, CG_ERR_CORRUPT);
 }
 
 }  // namespace
@@ -729,11 +578,6 @@ cudaError_t launch_decode(const DecParams& p, cudaStream_t stream) {
   if (err != cudaSuccess) return err;
   const uint64_t blocks = uint64_t(p.num_chunks) * p.L * 2 * p.units_per_slab;
   kern<<<unsigned(blocks), kThreads, sm.total, stream>>>(p);
-  if ((err = cudaGetLastError()) != cudaSuccess || !p.adjacent) return err;
-  const uint64_t work = uint64_t((p.C + kGroup - 1) / kGroup) * (p.H * p.D / 8);
-  const int per_slab = int((work + kChainThreads - 1) / kChainThreads);
-  chain_kernel<<<unsigned(uint64_t(p.num_chunks) * p.L * 2 * per_slab), kChainThreads, 0,
-                 stream>>>(p, per_slab);
   return cudaGetLastError();
 }
 
