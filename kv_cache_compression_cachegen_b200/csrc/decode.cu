@@ -65,6 +65,7 @@ struct DecSmem {
   uint32_t zs;      // f32 [2][2][D]  zero points and scales of the current and next head
   uint32_t rows;    // u64 [320]      destination row of each token (0: not written)
   uint32_t ok;      // u8  [320]      1 when the token's stream is being decoded
+  uint32_t gok;     // u8  [32]       1 when every stream of the anchor group is
   uint32_t single;  // i32 [H]        symbol of a one-symbol table, else -1
   uint32_t total;
 };
@@ -82,7 +83,8 @@ __host__ __device__ inline DecSmem dec_smem(int H, int D) {
   s.zs = al16(s.cum + 2u * kCumBuf);
   s.rows = al16(s.zs + 4u * uint32_t(D) * 4u);
   s.ok = al16(s.rows + uint32_t(kThreads) * 8u);
-  s.single = al16(s.ok + uint32_t(kThreads));
+  s.gok = al16(s.ok + uint32_t(kThreads));
+  s.single = al16(s.gok + uint32_t(kUnitGroups));
   s.total = al16(s.single + uint32_t(H) * 4u);
   return s;
 }
@@ -233,8 +235,12 @@ __device__ __forceinline__ void fill_table(uint32_t* tbl, CumBuf cb, int tid) {
 // the step inside the 64-byte ring and a step reads at most 16 bytes, which
 // may run into the mirror of slot 0.
 __device__ __forceinline__ uint32_t rans_step(uint32_t& x, uint32_t& ra, uint32_t& w,
-                                              const uint32_t* __restrict__ tbl) {
-  const uint32_t e = tbl[x & (kM - 1)];
+                                              uint32_t tbl_s) {
+  uint32_t e;
+  asm volatile("ld.shared.u32 %0, [%1];\n"
+               : "=r"(e)
+               : "r"(tbl_s + ((x & (kM - 1)) << 2))
+               : "memory");
   x = ((e >> 12) & (kM - 1)) * (x >> kProbBits) + (e & (kM - 1));
   asm volatile(
       "{\n\t"
@@ -258,12 +264,6 @@ __device__ __forceinline__ uint32_t ring_rebase(uint32_t ra, uint32_t rb) {
 // The symbols u (top bytes of four slot entries) as four bytes of one word.
 __device__ __forceinline__ uint32_t pack4(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t e3) {
   return __byte_perm(__byte_perm(e0, e1, 0x0073), __byte_perm(e2, e3, 0x0073), 0x5410);
-}
-
-// (float)(u - 127) for a symbol byte u: the bits 0x4B0000uu are the float
-// 2^23 + u, and subtracting 2^23 + 127 is exact.
-__device__ __forceinline__ float code_value(uint32_t u) {
-  return __fsub_rn(__uint_as_float(0x4B000000u | u), 8388735.0f);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
@@ -323,74 +323,141 @@ __device__ __forceinline__ uint16_t* dest_row(const DecParams& p, int chunk, int
 // Phase A for one head: decode D symbols of the thread's stream with the slot
 // table tb and leave their codes in the thread's row of the code buffer.
 __device__ __forceinline__ void decode_codes(uint32_t& x, uint32_t& p, uint32_t& ra,
-                                             uint32_t& w, Ring& r,
-                                             const uint32_t* __restrict__ tb,
-                                             uint8_t* __restrict__ crow, int D) {
+                                             uint32_t& w, Ring& r, uint32_t tb_s,
+                                             uint32_t crow_s, int D) {
   for (int d0 = 0; d0 < D; d0 += 8) {
     ring_issue(r, p);
     ring_wait_two_steps();
     ra = ring_rebase(ra, r.rb);
     const uint32_t ra0 = ra;
-    const uint32_t e0 = rans_step(x, ra, w, tb);
-    const uint32_t e1 = rans_step(x, ra, w, tb);
-    const uint32_t e2 = rans_step(x, ra, w, tb);
-    const uint32_t e3 = rans_step(x, ra, w, tb);
-    const uint32_t e4 = rans_step(x, ra, w, tb);
-    const uint32_t e5 = rans_step(x, ra, w, tb);
-    const uint32_t e6 = rans_step(x, ra, w, tb);
-    const uint32_t e7 = rans_step(x, ra, w, tb);
+    const uint32_t e0 = rans_step(x, ra, w, tb_s);
+    const uint32_t e1 = rans_step(x, ra, w, tb_s);
+    const uint32_t e2 = rans_step(x, ra, w, tb_s);
+    const uint32_t e3 = rans_step(x, ra, w, tb_s);
+    const uint32_t e4 = rans_step(x, ra, w, tb_s);
+    const uint32_t e5 = rans_step(x, ra, w, tb_s);
+    const uint32_t e6 = rans_step(x, ra, w, tb_s);
+    const uint32_t e7 = rans_step(x, ra, w, tb_s);
     p += (ra - ra0) >> 1;
-    *reinterpret_cast<uint2*>(crow + d0) = make_uint2(pack4(e0, e1, e2, e3), pack4(e4, e5, e6, e7));
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};\n" ::"r"(crow_s + uint32_t(d0)),
+                 "r"(pack4(e0, e1, e2, e3)), "r"(pack4(e4, e5, e6, e7))
+                 : "memory");
   }
 }
 
-// Phase B for one head: fp16 values from the codes.  Item (group g, channel
-// pair j): the anchor's pair, then the pair of each later token of the group.
-// A warp takes 32 consecutive pairs of one group (a "segment"), so each store
-// instruction writes 128 contiguous bytes of one token row; the segments are
-// dealt to the warps in turn.
-template <bool ADJ>
+// (float)(u - 127) for byte K of a word of codes: the bits 0x4B0000uu are the
+// float 2^23 + u, and subtracting 2^23 + 127 is exact.
+template <int K>
+__device__ __forceinline__ float code_byte(uint32_t w) {
+  return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | K)), 8388735.0f);
+}
+
+// Eight values a[k] + (float)q[k] * s[k] (round to nearest, no contraction)
+// of the eight codes in c, as fp16 (four words).
+template <bool SCALAR_S>
+__device__ __forceinline__ uint4 dequant8(const uint2 c, const float (&a)[8], const float* s,
+                                          float (&v)[8]) {
+  const uint32_t cw[2] = {c.x, c.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    v[4 * i + 0] = __fadd_rn(a[4 * i + 0], __fmul_rn(code_byte<0>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 0]));
+    v[4 * i + 1] = __fadd_rn(a[4 * i + 1], __fmul_rn(code_byte<1>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 1]));
+    v[4 * i + 2] = __fadd_rn(a[4 * i + 2], __fmul_rn(code_byte<2>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 2]));
+    v[4 * i + 3] = __fadd_rn(a[4 * i + 3], __fmul_rn(code_byte<3>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 3]));
+  }
+  return make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]), pack_half2(v[4], v[5]),
+                    pack_half2(v[6], v[7]));
+}
+
+// Where phase B writes: a flat destination (token t's row at row0 + t * HD)
+// or, for a paged pool, the per-token rows in shared memory (0: unmapped).
+struct RowMap {
+  uint16_t* row0;
+  uint64_t HD;
+  const uint64_t* rows;
+};
+
+template <bool PAGED>
+__device__ __forceinline__ uint16_t* row_of(const RowMap& m, int t) {
+  if (PAGED) return reinterpret_cast<uint16_t*>(m.rows[t]);
+  return m.row0 + uint64_t(t) * m.HD;
+}
+
+// Phase B for one head: fp16 values from the codes.  Item (group g, block b
+// of 8 channels): the anchor's 8 values a = zp + (float)c * scale, then the
+// same 8 channels of each later token of the group, a + (float)q * step
+// (format 2: each against the previous token's values), each row leaving as
+// one 16-byte store.  Consecutive lanes take consecutive blocks, so a warp's
+// stores cover whole row segments.
+// gok[g]: every stream of group g decodes; otherwise rows whose stream was
+// rejected are skipped (format 2: the rest of the chain too), and a group whose
+// anchor was rejected stays untouched.
+template <bool ADJ, bool PAGED>
 __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, uint32_t cstride,
-                                             const float* __restrict__ zh,
-                                             const uint64_t* __restrict__ rows,
-                                             const uint8_t* __restrict__ ok, int ngroups,
-                                             int ntok, int h, int D, float step, int warp,
-                                             int lane) {
-  const int P = D >> 1;                 // channel pairs per token row
-  const int S = (P + 31) >> 5;          // segments of 32 pairs per row
-  for (int wi = warp; wi < ngroups * S; wi += kWarps) {
-    const int g = S == 3 ? wi / 3 : wi >> (S >> 1);  // S is 1, 2, 3 or 4 (D <= 256)
-    const int j = (wi - g * S) * 32 + lane;
+                                             const float* __restrict__ zh, const RowMap& rm,
+                                             const uint8_t* __restrict__ ok,
+                                             const uint8_t* __restrict__ gok, int ngroups,
+                                             int ntok, int h, int D, float step, int tid,
+                                             int dq, int dr) {
+  const int B8 = D >> 3;
+  int g = tid / B8, b = tid - g * B8;  // item tid, then steps of kThreads = dq * B8 + dr items
+  for (; g < ngroups; g += dq, b += dr) {
+    if (b >= B8) {
+      b -= B8;
+      if (++g >= ngroups) break;
+    }
     const int t0 = g * kGroup;
-    if (j >= P || !ok[t0]) continue;  // past the row, or the anchor was rejected: untouched
-    const float2 z = *reinterpret_cast<const float2*>(zh + 2 * j);
-    const float2 sc = *reinterpret_cast<const float2*>(zh + D + 2 * j);
-    const uint32_t c = *reinterpret_cast<const uint16_t*>(codes + t0 * cstride + 2 * j);
-    float a0 = __fadd_rn(z.x, __fmul_rn(code_value(c & 0xFFu), sc.x));
-    float a1 = __fadd_rn(z.y, __fmul_rn(code_value(c >> 8), sc.y));
-    const uint32_t col = uint32_t(h * D + 2 * j);
-    uint16_t* r0 = reinterpret_cast<uint16_t*>(rows[t0]);
-    if (r0) *reinterpret_cast<uint32_t*>(r0 + col) = pack_half2(a0, a1);
-    const int tend = min(t0 + kGroup, ntok);
-    for (int t = t0 + 1; t < tend; ++t) {
-      if (!ok[t]) {
-        if (ADJ) break;  // the chain has lost a link: the rest of the group stays untouched
-        continue;
+    if (!ok[t0]) continue;
+    const int c0 = 8 * b;
+    float a[8], v[8];
+    {
+      const float4 z0 = *reinterpret_cast<const float4*>(zh + c0);
+      const float4 z1 = *reinterpret_cast<const float4*>(zh + c0 + 4);
+      const float4 s0 = *reinterpret_cast<const float4*>(zh + D + c0);
+      const float4 s1 = *reinterpret_cast<const float4*>(zh + D + c0 + 4);
+      const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+      const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const uint2 c = *reinterpret_cast<const uint2*>(codes + t0 * cstride + c0);
+      const uint4 hv = dequant8<false>(c, z, sc, a);
+      uint16_t* r = row_of<PAGED>(rm, t0);
+      if (!PAGED || r) *reinterpret_cast<uint4*>(r + h * D + c0) = hv;
+    }
+    const float st[1] = {step};
+    const int tend = min(kGroup, ntok - t0);
+    const uint8_t* cr = codes + t0 * cstride + c0;
+    if (gok[g]) {
+#pragma unroll
+      for (int r = 1; r < kGroup; ++r) {
+        if (r >= tend) break;
+        const uint2 q = *reinterpret_cast<const uint2*>(cr + r * cstride);
+        const uint4 hv = dequant8<true>(q, a, st, v);
+        uint16_t* row = row_of<PAGED>(rm, t0 + r);
+        if (!PAGED || row) *reinterpret_cast<uint4*>(row + h * D + c0) = hv;
+        if (ADJ) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) a[k] = v[k];
+        }
       }
-      const uint32_t q = *reinterpret_cast<const uint16_t*>(codes + t * cstride + 2 * j);
-      const float v0 = __fadd_rn(a0, __fmul_rn(code_value(q & 0xFFu), step));
-      const float v1 = __fadd_rn(a1, __fmul_rn(code_value(q >> 8), step));
-      uint16_t* rt = reinterpret_cast<uint16_t*>(rows[t]);
-      if (rt) *reinterpret_cast<uint32_t*>(rt + col) = pack_half2(v0, v1);
-      if (ADJ) {  // format 2: the next token's delta is taken against this value
-        a0 = v0;
-        a1 = v1;
+    } else {
+      for (int r = 1; r < tend; ++r) {
+        if (!ok[t0 + r]) {
+          if (ADJ) break;  // the chain has lost a link: the rest of the group stays untouched
+          continue;
+        }
+        const uint2 q = *reinterpret_cast<const uint2*>(cr + r * cstride);
+        const uint4 hv = dequant8<true>(q, a, st, v);
+        uint16_t* row = row_of<PAGED>(rm, t0 + r);
+        if (!PAGED || row) *reinterpret_cast<uint4*>(row + h * D + c0) = hv;
+        if (ADJ) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) a[k] = v[k];
+        }
       }
     }
   }
 }
 
-template <bool ADJ>
+template <bool ADJ, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_ok, s_n, s_bad;
@@ -432,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   const uint32_t cstride = codes_stride(D);
   uint64_t* rows = reinterpret_cast<uint64_t*>(smem + sm.rows);
   uint8_t* okf = smem + sm.ok;
+  uint8_t* gok = smem + sm.gok;
   int* single = reinterpret_cast<int*>(smem + sm.single);
   float* zs = reinterpret_cast<float*>(smem + sm.zs);  // [2][{zp, scale}][D]
   const int warp = tid >> 5, lane = tid & 31;
@@ -517,10 +585,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
       }
     }
   }
-  rows[tid] = orow;
+  if (PAGED) rows[tid] = orow;
   okf[tid] = active ? 1 : 0;
-  uint8_t* crow = codes + tid * cstride;
+  const uint32_t tbl_s = uint32_t(__cvta_generic_to_shared(tbl));
+  const uint32_t crow_s = uint32_t(__cvta_generic_to_shared(codes)) + uint32_t(tid) * cstride;
+  RowMap rm;
+  rm.HD = uint64_t(H) * D;
+  rm.rows = rows;
+  rm.row0 = PAGED ? nullptr : dest_row(p, chunk, slab, n, s_tstart, unit_t0);
+  const int dq = kThreads / (D >> 3), dr = kThreads - dq * (D >> 3);
   __syncthreads();
+  if (tid < ngroups) {  // whole-group flags for phase B's fast path
+    const int t0 = tid * kGroup, t1 = min(t0 + kGroup, ntok);
+    int all = 1;
+    for (int t = t0; t < t1; ++t) all &= okf[t];
+    gok[tid] = uint8_t(all);
+  }
 
   for (int h = 0; h < H; ++h) {
     // ---- phase A: the codes of head h
@@ -528,9 +608,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
       const int one = single[h];
       if (one >= 0) {  // a one-symbol table: the state stays put, no word is read
         const uint32_t cc = uint32_t(one) * 0x01010101u;
-        for (int d0 = 0; d0 < D; d0 += 8) *reinterpret_cast<uint2*>(crow + d0) = make_uint2(cc, cc);
+        for (int d0 = 0; d0 < D; d0 += 8)
+          asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(crow_s + uint32_t(d0)), "r"(cc)
+                       : "memory");
       } else {
-        decode_codes(x, pw, ra, w, ring, tbl + (h & 1) * kM, crow, D);
+        decode_codes(x, pw, ra, w, ring, tbl_s + uint32_t(h & 1) * kM * 4u, crow_s, D);
       }
     }
     // global loads for the next heads are issued before the barrier
@@ -550,8 +632,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
     __syncthreads();
     // ---- phase B: fp16 values of head h; the table, zero points and scales
     // of head h + 1, the compacted table of head h + 2
-    dequant_head<ADJ>(codes, cstride, zs + (h & 1) * 2 * D, rows, okf, ngroups, ntok, h, D, step,
-                      warp, lane);
+    dequant_head<ADJ, PAGED>(codes, cstride, zs + (h & 1) * 2 * D, rm, okf, gok, ngroups, ntok,
+                             h, D, step, tid, dq, dr);
     if (stage) {
       fill_table(tbl + ((h + 1) & 1) * kM, cum_buf(cumb + ((h + 1) & 1) * kCumBuf), tid);
       float* zn = zs + ((h + 1) & 1) * 2 * D;
@@ -572,7 +654,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
 
 cudaError_t launch_decode(const DecParams& p, cudaStream_t stream) {
   const DecSmem sm = dec_smem(p.H, p.D);
-  auto* kern = p.adjacent ? decode_kernel<true> : decode_kernel<false>;
+  auto* kern = p.adjacent ? (p.into == 2 ? decode_kernel<true, true> : decode_kernel<true, false>)
+                          : (p.into == 2 ? decode_kernel<false, true> : decode_kernel<false, false>);
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm.total));
   if (err != cudaSuccess) return err;

@@ -77,32 +77,50 @@ __host__ __device__ inline QSmem q_smem() {
   return s;
 }
 
+// Count the symbol of bracket word t = 0x4B400000 + u in the lane's column of
+// the shared histogram: hb is the column's address minus 0xA0000000, since
+// t << 7 = 0xA0000000 + 128 u modulo 2^32.
+__device__ __forceinline__ void hist_add(uint32_t hb, uint32_t t) {
+  asm volatile("red.shared.add.u32 [%0], 1;\n" ::"r"(hb + (t << 7)) : "memory");
+}
+
 // Exact quantisation of d = x - a by a step s with precomputed r = RN(1/s).
 // y = RN(d * r) is within 3 * 2^-24 |y| of RN(d / s) (three roundings of
 // relative size 2^-24).  The two values yc (1 - 2^-20) and yc (1 + 2^-20), yc
 // = y clamped to [-127, 127], bracket RN(d / s) (clamped alike) with room to
 // spare; each is rounded to an integer by one fused add of 1.5 * 2^23 + 127
-// (ulp 1 there).  When both give the same integer, no half-integer lies
-// between them, so round-half-away-from-zero of RN(d / s) gives that integer
-// too, and the low byte of the sum is u = q + 127.  `ok` turns false when the
-// two differ (a value near a half-integer) or |y| >= 2^22 (a huge or
-// non-finite input); the caller then takes the definition itself.
-__device__ __forceinline__ uint32_t quant_fast(float d, float r, bool& ok) {
+// (ulp 1 there), giving the word t = 0x4B400000 + u.  When both give the same
+// integer, no half-integer lies between them, so round-half-away-from-zero of
+// RN(d / s) gives that integer too.  For a row of 8 values the caller ORs
+// t1 ^ t2 into `diff` and takes the definition (quant_exact) for the whole row
+// when any bit differs.  A quotient that is not finite (an infinite or NaN
+// input) cannot be bracketed: y * 0 turns `nanacc` into NaN, and the caller
+// reports the input.  Every finite y is clamped into [-127, 127], where the
+// bracket holds (a huge quotient clamps to +-127 on both paths).
+__device__ __forceinline__ uint32_t quant_bits(float d, float r, uint32_t& diff, float& nanacc) {
   const float y = __fmul_rn(d, r);
+  nanacc = __fmaf_rn(y, 0.0f, nanacc);
   const float yc = fminf(fmaxf(y, -127.0f), 127.0f);
-  const float t1 = __fmaf_rn(yc, 1.0f + 0x1p-20f, 12583039.0f);
-  const float t2 = __fmaf_rn(yc, 1.0f - 0x1p-20f, 12583039.0f);
-  ok = ok && (__float_as_uint(t1) == __float_as_uint(t2)) && (fabsf(y) < 0x1p22f);
-  return __float_as_uint(t1) & 0xFFu;
+  const uint32_t t1 = __float_as_uint(__fmaf_rn(yc, 1.0f + 0x1p-20f, 12583039.0f));
+  const uint32_t t2 = __float_as_uint(__fmaf_rn(yc, 1.0f - 0x1p-20f, 12583039.0f));
+  diff |= t1 ^ t2;
+  return t1;
 }
 
 // The definition itself: u = clamp(roundf(RN(RN(x - a) / s)), -127, 127) + 127,
-// with s == 0 (a constant anchor channel) giving code 0.
+// with s == 0 (a constant anchor channel) giving code 0; returned in the form
+// of a bracket word, 0x4B400000 + u.
 __device__ __forceinline__ uint32_t quant_exact(float x, float a, float s) {
-  if (s == 0.0f) return 127u;
+  if (s == 0.0f) return 0x4B400000u + 127u;
   const float y = __fdiv_rn(__fsub_rn(x, a), s);
   const float r = fminf(fmaxf(roundf(y), -127.0f), 127.0f);
-  return uint32_t(int(r) + 127);
+  return 0x4B400000u + uint32_t(int(r) + 127);
+}
+
+// (float)q of a bracket word t = 0x4B400000 + u: t is the float 2^23 + 2^22 + u,
+// and subtracting 2^23 + 2^22 + 127 is exact.
+__device__ __forceinline__ float code_of(uint32_t t) {
+  return __fsub_rn(__uint_as_float(t), 12583039.0f);
 }
 
 __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) {
@@ -257,7 +275,7 @@ __device__ __forceinline__ void unpack8(const uint4 rv, float (&x)[8]) {
 // adjacent tokens) instead of the group's anchor; a lane walks its group's
 // rows in order, so the running reconstruction stays in its registers.
 template <int NL, bool ADJ>
-__global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, const int mode) {
+__global__ void __launch_bounds__(kQThreads, NL == 1 ? 3 : 2) quant_kernel(const EncParams p, const int mode) {
   static_assert(!(ADJ && NL != 1), "format 2 is encoded one level at a time");
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -387,9 +405,10 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
   }
   __syncthreads();
 
-  // ---- Phase B: quantise group by group.  Each lane loads the ten rows of its
-  // group for its 8 channels; the rows of the warp's next group set are loaded
-  // before the current set is quantised.
+  // ---- Phase B: quantise group by group.  A lane walks the ten rows of its
+  // group for its 8 channels (one 16-byte load per row), then the ten rows of
+  // its next group set; the loads run five rows ahead in a register ring,
+  // across the boundary between group sets.
   float step[NL], rstep[NL];
 #pragma unroll
   for (int j = 0; j < NL; ++j) {
@@ -399,89 +418,112 @@ __global__ void __launch_bounds__(kQThreads, 2) quant_kernel(const EncParams p, 
   const uint64_t symo = ((uint64_t(chunk) * L * 2 + slab) * H + h) * uint64_t(D / 16) * C * 16 +
                         (ql.c >> 1) * uint64_t(C) * 16 + (ql.c & 1) * 8;
   auto symc_of = [&](int j) { return (NL == 1 ? p.sym : p.lsym[j]) + symo; };
-  auto put_syms = [&](int j, int tok, const uint32_t (&u)[8]) {
+  // Histogram counter of symbol u for this lane: hist + 4 lane + 128 u (bank =
+  // lane).  A bracket word is t = 0x4B400000 + u (see quant_bits), so
+  // t << 7 = 0xA0000000 + 128 u modulo 2^32 and the address is one shift-add.
+  const uint32_t hist_t = uint32_t(__cvta_generic_to_shared(hist)) + 4u * lane - 0xA0000000u;
+  auto put_syms = [&](int j, int tok, uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
+                      uint32_t t4, uint32_t t5, uint32_t t6, uint32_t t7) {
     if (want_hist) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) atomicAdd(&hist[(j * kAlphabet + u[k]) * 32 + lane], 1u);
+      const uint32_t hb = hist_t + (uint32_t(j * kAlphabet) << 7);
+      hist_add(hb, t0);
+      hist_add(hb, t1);
+      hist_add(hb, t2);
+      hist_add(hb, t3);
+      hist_add(hb, t4);
+      hist_add(hb, t5);
+      hist_add(hb, t6);
+      hist_add(hb, t7);
     }
     if (want_sym)
       *reinterpret_cast<uint2*>(symc_of(j) + uint64_t(tok) * 16) =
-          make_uint2(u[0] | (u[1] << 8) | (u[2] << 16) | (u[3] << 24),
-                     u[4] | (u[5] << 8) | (u[6] << 16) | (u[7] << 24));
+          make_uint2(__byte_perm(__byte_perm(t0, t1, 0x0040), __byte_perm(t2, t3, 0x0040), 0x5410),
+                     __byte_perm(__byte_perm(t4, t5, 0x0040), __byte_perm(t6, t7, 0x0040), 0x5410));
   };
-  uint4 nx[kGroup];
-  auto load_set = [&](int gs, uint4 (&v)[kGroup]) {
+  // rows of group set gs available to this lane (0 past the chunk's groups)
+  auto set_rows = [&](int gs) {
     const int g = gs * ql.rpw + ql.r;
-    const int tg = g * kGroup;
-#pragma unroll
-    for (int j = 0; j < kGroup; ++j)
-      v[j] = ql.on && gs < nsets && g < Gn && tg + j < n
-                 ? __ldg(reinterpret_cast<const uint4*>(col + uint64_t(tg + j) * rs + ch))
-                 : make_uint4(0, 0, 0, 0);
+    return (ql.on && gs < nsets && g < Gn) ? min(kGroup, n - g * kGroup) : 0;
   };
-  load_set(warp, nx);
+  auto set_ptr = [&](int gs) {
+    return col + uint64_t(gs * ql.rpw + ql.r) * kGroup * rs + ch;
+  };
+  float nanacc = 0.0f;  // becomes NaN once a quotient is not finite
+  constexpr int kAhead = 5;  // ring depth (kGroup is a multiple of it)
+  uint4 ring[kAhead];
+  int ntok = set_rows(warp);
+  const uint16_t* rp = set_ptr(warp);
+#pragma unroll
+  for (int j = 0; j < kAhead; ++j)
+    ring[j] = j < ntok ? __ldg(reinterpret_cast<const uint4*>(rp + uint64_t(j) * rs))
+                       : make_uint4(0, 0, 0, 0);
   for (int gs = warp; gs < nsets; gs += kQWarps) {
-    uint4 cur[kGroup];
-#pragma unroll
-    for (int j = 0; j < kGroup; ++j) cur[j] = nx[j];
-    load_set(gs + kQWarps, nx);
-    const int g = gs * ql.rpw + ql.r;
-    if (!(ql.on && g < Gn)) continue;
-    const int tg = g * kGroup;
-    const int ntok = min(kGroup, n - tg);
-    // anchor: code against (zp, scale), reconstructed value a
+    const int tg = (gs * ql.rpw + ql.r) * kGroup;
+    const int ntok_next = set_rows(gs + kQWarps);
+    const uint16_t* rpn = set_ptr(gs + kQWarps);
     float a[8];
-    {
-      float x[8], zc[8], scc[8], rc[8];
-      unpack8(cur[0], x);
 #pragma unroll
-      for (int k = 0; k < 8; k += 4) {  // this lane's channels, from shared memory
-        const float4 za = *reinterpret_cast<const float4*>(zp + ch + k);
-        const float4 sa = *reinterpret_cast<const float4*>(sc + ch + k);
-        const float4 ra = *reinterpret_cast<const float4*>(rcp + ch + k);
-        zc[k] = za.x; zc[k + 1] = za.y; zc[k + 2] = za.z; zc[k + 3] = za.w;
-        scc[k] = sa.x; scc[k + 1] = sa.y; scc[k + 2] = sa.z; scc[k + 3] = sa.w;
-        rc[k] = ra.x; rc[k + 1] = ra.y; rc[k + 2] = ra.z; rc[k + 3] = ra.w;
+    for (int r = 0; r < kGroup; ++r) {
+      const uint4 cur = ring[r % kAhead];
+      // refill the slot: row r + 5 of this set, or row r - 5 of the next one
+      if (r + kAhead < kGroup) {
+        ring[r % kAhead] = r + kAhead < ntok
+            ? __ldg(reinterpret_cast<const uint4*>(rp + uint64_t(r + kAhead) * rs))
+            : make_uint4(0, 0, 0, 0);
+      } else {
+        ring[r % kAhead] = r + kAhead - kGroup < ntok_next
+            ? __ldg(reinterpret_cast<const uint4*>(rpn + uint64_t(r + kAhead - kGroup) * rs))
+            : make_uint4(0, 0, 0, 0);
       }
-      uint32_t u[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        if (!isfinite(x[k])) nonfinite = true;
-        bool ok = true;
-        u[k] = quant_fast(__fsub_rn(x[k], zc[k]), rc[k], ok);
-        if (!ok) u[k] = quant_exact(x[k], zc[k], scc[k]);
-        a[k] = __fadd_rn(zc[k], __fmul_rn(float(int(u[k]) - 127), scc[k]));
-      }
-#pragma unroll
-      for (int j = 0; j < NL; ++j) put_syms(j, tg, u);
-    }
-#pragma unroll
-    for (int r = 1; r < kGroup; ++r) {
-      if (r >= ntok) break;
+      if (r >= ntok) continue;
       float x[8];
-      unpack8(cur[r], x);
+      unpack8(cur, x);
+      if (r == 0) {
+        // anchor: code against (zp, scale), reconstructed value a
+        float zc[8], scc[8], rc[8];
 #pragma unroll
-      for (int j = 0; j < NL; ++j) {
-        bool ok = true;
-        uint32_t u[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) u[k] = quant_fast(__fsub_rn(x[k], a[k]), rstep[j], ok);
-        if (!ok) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            if (!isfinite(x[k])) nonfinite = true;
-            u[k] = quant_exact(x[k], a[k], step[j]);
-          }
+        for (int k = 0; k < 8; k += 4) {  // this lane's channels, from shared memory
+          const float4 za = *reinterpret_cast<const float4*>(zp + ch + k);
+          const float4 sa = *reinterpret_cast<const float4*>(sc + ch + k);
+          const float4 ra = *reinterpret_cast<const float4*>(rcp + ch + k);
+          zc[k] = za.x; zc[k + 1] = za.y; zc[k + 2] = za.z; zc[k + 3] = za.w;
+          scc[k] = sa.x; scc[k + 1] = sa.y; scc[k + 2] = sa.z; scc[k + 3] = sa.w;
+          rc[k] = ra.x; rc[k + 1] = ra.y; rc[k + 2] = ra.z; rc[k + 3] = ra.w;
         }
-        put_syms(j, tg + r, u);
-        if (ADJ) {  // the next row's reference: this row's reconstruction
+        uint32_t t[8], diff = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) t[k] = quant_bits(__fsub_rn(x[k], zc[k]), rc[k], diff, nanacc);
+        if (diff) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) t[k] = quant_exact(x[k], zc[k], scc[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[k] = __fadd_rn(zc[k], __fmul_rn(code_of(t[k]), scc[k]));
+#pragma unroll
+        for (int j = 0; j < NL; ++j) put_syms(j, tg, t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < NL; ++j) {
+          uint32_t t[8], diff = 0;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            a[k] = __fadd_rn(a[k], __fmul_rn(float(int(u[k]) - 127), step[j]));
+            t[k] = quant_bits(__fsub_rn(x[k], a[k]), rstep[j], diff, nanacc);
+          if (diff) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t[k] = quant_exact(x[k], a[k], step[j]);
+          }
+          put_syms(j, tg + r, t[0], t[1], t[2], t[3], t[4], t[5], t[6], t[7]);
+          if (ADJ) {  // the next row's reference: this row's reconstruction
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a[k] = __fadd_rn(a[k], __fmul_rn(code_of(t[k]), step[j]));
+          }
         }
       }
     }
+    ntok = ntok_next;
+    rp = rpn;
   }
+  if (nanacc != nanacc) nonfinite = true;
   __syncthreads();
   if (nonfinite) set_status(p.status, CG_ERR_NONFINITE);
 
