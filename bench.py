@@ -34,16 +34,16 @@ WORKLOAD = dict(name="llama2_7b", L=32, H=32, D=128, T=10752, C=1536, seed=2, rh
 METRIC = "cg_decode / cg_encode GB/s (fp16 KV) on 1 B200, % of HBM roofline, compression ratio"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) per fp16 value of decode_kernel from one ncu capture
-# of the current kernel (103.9 MB read + 352.8 MB written for a Mistral-7B-shaped
-# 32x2x3072x8x128 case = 201,326,592 values); the bench reports it scaled by its
-# own value count.  The capture ends with up to one L2 (126 MB) of written lines
-# not yet in DRAM, so this slightly undercounts.
-DECODE_DRAM_BYTES_PER_VALUE = (103_913_472 + 352_763_136) / 201_326_592
+# of the current kernel on a Llama-2-7B-shaped case (32x2x3072x32x128 =
+# 805,306,368 values: 342.2 MB read + 1,552.9 MB written); the bench reports it
+# scaled by its own value count.  The capture ends with up to one L2 (126 MB)
+# of written lines not yet in DRAM, so this slightly undercounts.
+DECODE_DRAM_BYTES_PER_VALUE = (342_183_680 + 1_552_913_000) / 805_306_368
 # Shared-memory wavefronts per warp-symbol of decode_kernel from the same
-# capture (48,259,107 wavefronts for 201,326,592 symbols): the random slot-table
-# lookups of 32 streams cost about four, the word refills, the reconstructed
-# anchors and the table fills the rest.  An SM serves one wavefront per clock.
-DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL = 48_259_107 / (201_326_592 / 32)
+# capture (181,248,933 wavefronts for 805,306,368 symbols): the random slot-table
+# lookups of 32 streams cost about four, the word refills, the code stores and
+# loads and the table fills the rest.  An SM serves one wavefront per clock.
+DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL = 181_248_933 / (805_306_368 / 32)
 
 
 def smem_ceiling(symbols: int, ms: float, sm_mhz, sms: int):
@@ -56,7 +56,7 @@ def smem_ceiling(symbols: int, ms: float, sm_mhz, sms: int):
     return {"bound": "smem", "achieved": round(achieved / 1e9, 1), "peak": round(peak / 1e9, 1),
             "unit": "G wavefronts/s", "frac": round(achieved / peak, 4),
             "wavefronts_per_warp_symbol": round(DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL, 2),
-            "source": "ncu wavefronts per warp-symbol of a 3,072-token Mistral-7B-shaped "
+            "source": "ncu wavefronts per warp-symbol of a 3,072-token Llama-2-7B-shaped "
                       "capture; peak = SMs x sampled SM clock"}
 
 
@@ -363,7 +363,7 @@ def run_ours(args):
                          "frac": round(dec_frac, 4),
                          "traffic": int(DECODE_DRAM_BYTES_PER_VALUE * (fp16_bytes // 2)),
                          "traffic_source": "ncu dram bytes per value of a 3,072-token "
-                                           "Mistral-7B-shaped capture, scaled by values",
+                                           "Llama-2-7B-shaped capture, scaled by values",
                          "algorithmic_bytes": alg},
             "gpu_launches": 5 * args.steps,
             "clocks": clocks,
