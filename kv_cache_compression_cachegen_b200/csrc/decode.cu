@@ -18,16 +18,17 @@
 //            the only shared-memory traffic is the slot-table lookup, the word
 //            refill and one 8-byte code store per 8 symbols.
 //   phase B  the threads turn the codes of head h into fp16.  A work item is
-//            (anchor group g, channel pair): the anchor value
+//            (anchor group g, 8 channels): the anchor's values
 //            a = zp + (float)c * scale, then the nine deltas a + (float)q * step
 //            (format 2: each delta against the previous token's value), all
 //            fp32 with IEEE round-to-nearest adds and multiplies (no
-//            contraction), stored as fp16 pairs; the 32 lanes of a warp take
-//            32 consecutive pairs of one token row, so every store instruction
-//            writes whole 32-byte sectors.  Meanwhile the slot table of head
-//            h + 1 is built and the zero points / scales of head h + 1 staged.
+//            contraction), each row's 8 values leaving as one 16-byte store;
+//            consecutive lanes take consecutive channel blocks, so a warp's
+//            stores cover whole row segments.  Meanwhile the slot table is
+//            rebuilt for head h + 1 (phase A of head h no longer reads it) and
+//            the zero points / scales of head h + 1 are staged.
 //
-// A __syncthreads separates the phases.  Anchors get no special treatment in
+// A __syncthreads separates the phases (two per head).  Anchors get no special treatment in
 // phase A, and the reconstructed anchors never leave the registers of the
 // phase-B item, so the work of a head is spread evenly over the CTA.
 //
@@ -57,7 +58,8 @@ constexpr uint32_t kRingStride = kRingBytes + 16;       // + a copy of slot 0 af
 
 // Dynamic shared memory layout (byte offsets), a function of H and D.
 struct DecSmem {
-  uint32_t tbl;     // u32 [2][4096]  slot tables, packed (u << 24) | (f << 12) | (slot - cum)
+  uint32_t tbl;     // u32 [4096]     slot table of the current head, packed
+                    //                (u << 24) | (f << 12) | (slot - cum)
   uint32_t codes;   // u8  [320][D + 8]  symbols u of the current head, one row per token
   uint32_t ring;    // u8  [320][80]  per-thread word rings: 4 slots + a mirror of slot 0
   uint32_t cum;     // [2] x {u16 pcum[257], u8 psym[256], i32 nz}: compacted tables of
@@ -77,7 +79,7 @@ __host__ __device__ inline uint32_t codes_stride(int D) { return uint32_t(D) + 8
 __host__ __device__ inline DecSmem dec_smem(int H, int D) {
   DecSmem s;
   s.tbl = 0;
-  s.codes = s.tbl + 2u * 4096u * 4u;
+  s.codes = s.tbl + 4096u * 4u;
   s.ring = al16(s.codes + uint32_t(kThreads) * codes_stride(D));
   s.cum = al16(s.ring + uint32_t(kThreads) * kRingStride);
   s.zs = al16(s.cum + 2u * kCumBuf);
@@ -426,13 +428,20 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
     const int tend = min(kGroup, ntok - t0);
     const uint8_t* cr = codes + t0 * cstride + c0;
     if (gok[g]) {
+      // flat destinations: the rows of consecutive tokens are HD values apart
+      uint16_t* fr = PAGED ? nullptr : row_of<false>(rm, t0) + (h * D + c0);
 #pragma unroll
       for (int r = 1; r < kGroup; ++r) {
         if (r >= tend) break;
         const uint2 q = *reinterpret_cast<const uint2*>(cr + r * cstride);
         const uint4 hv = dequant8<true>(q, a, st, v);
-        uint16_t* row = row_of<PAGED>(rm, t0 + r);
-        if (!PAGED || row) *reinterpret_cast<uint4*>(row + h * D + c0) = hv;
+        if (PAGED) {
+          uint16_t* row = row_of<true>(rm, t0 + r);
+          if (row) *reinterpret_cast<uint4*>(row + h * D + c0) = hv;
+        } else {
+          fr += rm.HD;
+          *reinterpret_cast<uint4*>(fr) = hv;
+        }
         if (ADJ) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) a[k] = v[k];
@@ -612,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
           asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(crow_s + uint32_t(d0)), "r"(cc)
                        : "memory");
       } else {
-        decode_codes(x, pw, ra, w, ring, tbl_s + uint32_t(h & 1) * kM * 4u, crow_s, D);
+        decode_codes(x, pw, ra, w, ring, tbl_s, crow_s, D);
       }
     }
     // global loads for the next heads are issued before the barrier
@@ -635,7 +644,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
     dequant_head<ADJ, PAGED>(codes, cstride, zs + (h & 1) * 2 * D, rm, okf, gok, ngroups, ntok,
                              h, D, step, tid, dq, dr);
     if (stage) {
-      fill_table(tbl + ((h + 1) & 1) * kM, cum_buf(cumb + ((h + 1) & 1) * kCumBuf), tid);
+      // phase A of head h is over: the table is rebuilt for head h + 1
+      fill_table(tbl, cum_buf(cumb + ((h + 1) & 1) * kCumBuf), tid);
       float* zn = zs + ((h + 1) & 1) * 2 * D;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
