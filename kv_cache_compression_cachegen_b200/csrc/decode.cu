@@ -74,7 +74,12 @@ struct DecSmem {
 
 __host__ __device__ inline uint32_t al16(uint32_t v) { return (v + 15u) & ~15u; }
 
-__host__ __device__ inline uint32_t codes_stride(int D) { return uint32_t(D) + 8u; }
+// A head is decoded in kSlices slices of D / kSlices channels (two phases
+// each), so the code buffer holds one slice: that keeps a CTA's shared memory
+// small enough for three CTAs per SM.
+constexpr int kSlices = 2;
+
+__host__ __device__ inline uint32_t codes_stride(int D) { return uint32_t(D / kSlices) + 8u; }
 
 __host__ __device__ inline DecSmem dec_smem(int H, int D) {
   DecSmem s;
@@ -399,9 +404,9 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
                                              const float* __restrict__ zh, const RowMap& rm,
                                              const uint8_t* __restrict__ ok,
                                              const uint8_t* __restrict__ gok, int ngroups,
-                                             int ntok, int h, int D, float step, int tid,
-                                             int dq, int dr) {
-  const int B8 = D >> 3;
+                                             int ntok, int h, int D, int cbase, int DS,
+                                             float step, int tid, int dq, int dr) {
+  const int B8 = DS >> 3;
   int g = tid / B8, b = tid - g * B8;  // item tid, then steps of kThreads = dq * B8 + dr items
   for (; g < ngroups; g += dq, b += dr) {
     if (b >= B8) {
@@ -410,26 +415,27 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
     }
     const int t0 = g * kGroup;
     if (!ok[t0]) continue;
-    const int c0 = 8 * b;
+    const int c0 = 8 * b;      // column in the slice's code rows
+    const int cz = cbase + c0;  // channel in the head
     float a[8], v[8];
     {
-      const float4 z0 = *reinterpret_cast<const float4*>(zh + c0);
-      const float4 z1 = *reinterpret_cast<const float4*>(zh + c0 + 4);
-      const float4 s0 = *reinterpret_cast<const float4*>(zh + D + c0);
-      const float4 s1 = *reinterpret_cast<const float4*>(zh + D + c0 + 4);
+      const float4 z0 = *reinterpret_cast<const float4*>(zh + cz);
+      const float4 z1 = *reinterpret_cast<const float4*>(zh + cz + 4);
+      const float4 s0 = *reinterpret_cast<const float4*>(zh + D + cz);
+      const float4 s1 = *reinterpret_cast<const float4*>(zh + D + cz + 4);
       const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
       const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
       const uint2 c = *reinterpret_cast<const uint2*>(codes + t0 * cstride + c0);
       const uint4 hv = dequant8<false>(c, z, sc, a);
       uint16_t* r = row_of<PAGED>(rm, t0);
-      if (!PAGED || r) *reinterpret_cast<uint4*>(r + h * D + c0) = hv;
+      if (!PAGED || r) *reinterpret_cast<uint4*>(r + h * D + cz) = hv;
     }
     const float st[1] = {step};
     const int tend = min(kGroup, ntok - t0);
     const uint8_t* cr = codes + t0 * cstride + c0;
     if (gok[g]) {
       // flat destinations: the rows of consecutive tokens are HD values apart
-      uint16_t* fr = PAGED ? nullptr : row_of<false>(rm, t0) + (h * D + c0);
+      uint16_t* fr = PAGED ? nullptr : row_of<false>(rm, t0) + (h * D + cz);
 #pragma unroll
       for (int r = 1; r < kGroup; ++r) {
         if (r >= tend) break;
@@ -437,7 +443,7 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
         const uint4 hv = dequant8<true>(q, a, st, v);
         if (PAGED) {
           uint16_t* row = row_of<true>(rm, t0 + r);
-          if (row) *reinterpret_cast<uint4*>(row + h * D + c0) = hv;
+          if (row) *reinterpret_cast<uint4*>(row + h * D + cz) = hv;
         } else {
           fr += rm.HD;
           *reinterpret_cast<uint4*>(fr) = hv;
@@ -456,7 +462,7 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
         const uint2 q = *reinterpret_cast<const uint2*>(cr + r * cstride);
         const uint4 hv = dequant8<true>(q, a, st, v);
         uint16_t* row = row_of<PAGED>(rm, t0 + r);
-        if (!PAGED || row) *reinterpret_cast<uint4*>(row + h * D + c0) = hv;
+        if (!PAGED || row) *reinterpret_cast<uint4*>(row + h * D + cz) = hv;
         if (ADJ) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) a[k] = v[k];
@@ -467,7 +473,7 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
 }
 
 template <bool ADJ, bool PAGED>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) {
+__global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int s_ok, s_n, s_bad;
   __shared__ long long s_tstart;
@@ -602,7 +608,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   rm.HD = uint64_t(H) * D;
   rm.rows = rows;
   rm.row0 = PAGED ? nullptr : dest_row(p, chunk, slab, n, s_tstart, unit_t0);
-  const int dq = kThreads / (D >> 3), dr = kThreads - dq * (D >> 3);
+  const int DS = D / kSlices;  // channels of a slice (a multiple of 8)
+  const int dq = kThreads / (DS >> 3), dr = kThreads - dq * (DS >> 3);
   __syncthreads();
   if (tid < ngroups) {  // whole-group flags for phase B's fast path
     const int t0 = tid * kGroup, t1 = min(t0 + kGroup, ntok);
@@ -612,49 +619,53 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecParams p) 
   }
 
   for (int h = 0; h < H; ++h) {
-    // ---- phase A: the codes of head h
-    if (active) {
-      const int one = single[h];
-      if (one >= 0) {  // a one-symbol table: the state stays put, no word is read
-        const uint32_t cc = uint32_t(one) * 0x01010101u;
-        for (int d0 = 0; d0 < D; d0 += 8)
-          asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(crow_s + uint32_t(d0)), "r"(cc)
-                       : "memory");
-      } else {
-        decode_codes(x, pw, ra, w, ring, tbl_s, crow_s, D);
+    for (int sl = 0; sl < kSlices; ++sl) {
+      const bool last = sl == kSlices - 1;
+      // ---- phase A: the codes of slice sl of head h
+      if (active) {
+        const int one = single[h];
+        if (one >= 0) {  // a one-symbol table: the state stays put, no word is read
+          const uint32_t cc = uint32_t(one) * 0x01010101u;
+          for (int d0 = 0; d0 < DS; d0 += 8)
+            asm volatile("st.shared.v2.u32 [%0], {%1, %1};\n" ::"r"(crow_s + uint32_t(d0)), "r"(cc)
+                         : "memory");
+        } else {
+          decode_codes(x, pw, ra, w, ring, tbl_s, crow_s, DS);
+        }
       }
-    }
-    // global loads for the next heads are issued before the barrier
-    const bool scan_warp = h + 2 < H && warp == h % kWarps;
-    uint4 fq = make_uint4(0, 0, 0, 0);
-    if (scan_warp) fq = __ldg(reinterpret_cast<const uint4*>(freq + (h + 2) * 256) + lane);
-    float zv[2] = {0.0f, 0.0f};
-    const bool stage = h + 1 < H;
-    if (stage) {
+      // global loads for the next heads are issued before the barrier
+      const bool scan_warp = last && h + 2 < H && warp == h % kWarps;
+      uint4 fq = make_uint4(0, 0, 0, 0);
+      if (scan_warp) fq = __ldg(reinterpret_cast<const uint4*>(freq + (h + 2) * 256) + lane);
+      float zv[2] = {0.0f, 0.0f};
+      const bool stage = last && h + 1 < H;
+      if (stage) {
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int i = tid + j * kThreads;
-        if (i < 2 * D)
-          zv[j] = i < D ? __ldg(zp_sec + (h + 1) * D + i) : __ldg(sc_sec + (h + 1) * D + (i - D));
+        for (int j = 0; j < 2; ++j) {
+          const int i = tid + j * kThreads;
+          if (i < 2 * D)
+            zv[j] = i < D ? __ldg(zp_sec + (h + 1) * D + i) : __ldg(sc_sec + (h + 1) * D + (i - D));
+        }
       }
-    }
-    __syncthreads();
-    // ---- phase B: fp16 values of head h; the table, zero points and scales
-    // of head h + 1, the compacted table of head h + 2
-    dequant_head<ADJ, PAGED>(codes, cstride, zs + (h & 1) * 2 * D, rm, okf, gok, ngroups, ntok,
-                             h, D, step, tid, dq, dr);
-    if (stage) {
-      // phase A of head h is over: the table is rebuilt for head h + 1
-      fill_table(tbl, cum_buf(cumb + ((h + 1) & 1) * kCumBuf), tid);
-      float* zn = zs + ((h + 1) & 1) * 2 * D;
+      __syncthreads();
+      // ---- phase B: fp16 values of slice sl of head h; after the last slice
+      // the table, zero points and scales of head h + 1 and the compacted
+      // table of head h + 2
+      dequant_head<ADJ, PAGED>(codes, cstride, zs + (h & 1) * 2 * D, rm, okf, gok, ngroups, ntok,
+                               h, D, sl * DS, DS, step, tid, dq, dr);
+      if (stage) {
+        // phase A of head h is over: the table is rebuilt for head h + 1
+        fill_table(tbl, cum_buf(cumb + ((h + 1) & 1) * kCumBuf), tid);
+        float* zn = zs + ((h + 1) & 1) * 2 * D;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int i = tid + j * kThreads;
-        if (i < 2 * D) zn[i] = zv[j];
+        for (int j = 0; j < 2; ++j) {
+          const int i = tid + j * kThreads;
+          if (i < 2 * D) zn[i] = zv[j];
+        }
       }
+      if (scan_warp) cum_compact(fq, cum_buf(cumb + (h & 1) * kCumBuf), lane);
+      __syncthreads();
     }
-    if (scan_warp) cum_compact(fq, cum_buf(cumb + (h & 1) * kCumBuf), lane);
-    __syncthreads();
   }
   ring_wait_all();
   if (active && (x != kRansL || pw != pend)) set_status(p.status, CG_ERR_CORRUPT);
