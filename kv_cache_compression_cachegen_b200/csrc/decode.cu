@@ -352,28 +352,35 @@ __device__ __forceinline__ void decode_codes(uint32_t& x, uint32_t& p, uint32_t&
   }
 }
 
-// (float)(u - 127) for byte K of a word of codes: the bits 0x4B0000uu are the
-// float 2^23 + u, and subtracting 2^23 + 127 is exact.
+// (float)(u - 127) for bytes K and K + 1 of a word of codes: the bits
+// 0x4B0000uu are the float 2^23 + u, and subtracting 2^23 + 127 is exact.
 template <int K>
-__device__ __forceinline__ float code_byte(uint32_t w) {
-  return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | K)), 8388735.0f);
+__device__ __forceinline__ float2 code_pair(uint32_t w) {
+  const float2 biased = make_float2(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | K)),
+                                    __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u | (K + 1))));
+  return add2_rn(biased, make_float2(-8388735.0f, -8388735.0f));
 }
 
-// Eight values a[k] + (float)q[k] * s[k] (round to nearest, no contraction)
-// of the eight codes in c, as fp16 (four words).
+// Eight values a[k] + (float)q[k] * s[k] of the eight codes in c, as fp16 (four
+// words): codes and products two channels per packed instruction, the final
+// adds one channel at a time.
 template <bool SCALAR_S>
-__device__ __forceinline__ uint4 dequant8(const uint2 c, const float (&a)[8], const float* s,
-                                          float (&v)[8]) {
+__device__ __forceinline__ uint4 dequant8(const uint2 c, const float2 (&a)[4], const float2* s,
+                                          float2 (&v)[4]) {
   const uint32_t cw[2] = {c.x, c.y};
+  uint32_t h[4];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    v[4 * i + 0] = __fadd_rn(a[4 * i + 0], __fmul_rn(code_byte<0>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 0]));
-    v[4 * i + 1] = __fadd_rn(a[4 * i + 1], __fmul_rn(code_byte<1>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 1]));
-    v[4 * i + 2] = __fadd_rn(a[4 * i + 2], __fmul_rn(code_byte<2>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 2]));
-    v[4 * i + 3] = __fadd_rn(a[4 * i + 3], __fmul_rn(code_byte<3>(cw[i]), SCALAR_S ? s[0] : s[4 * i + 3]));
+    const float2 q0 = code_pair<0>(cw[i]);
+    const float2 q1 = code_pair<2>(cw[i]);
+    const float2 p0 = mul2_rn(q0, SCALAR_S ? s[0] : s[2 * i + 0]);
+    const float2 p1 = mul2_rn(q1, SCALAR_S ? s[0] : s[2 * i + 1]);
+    v[2 * i + 0] = make_float2(__fadd_rn(a[2 * i + 0].x, p0.x), __fadd_rn(a[2 * i + 0].y, p0.y));
+    v[2 * i + 1] = make_float2(__fadd_rn(a[2 * i + 1].x, p1.x), __fadd_rn(a[2 * i + 1].y, p1.y));
+    h[2 * i + 0] = pack_half2(v[2 * i + 0].x, v[2 * i + 0].y);
+    h[2 * i + 1] = pack_half2(v[2 * i + 1].x, v[2 * i + 1].y);
   }
-  return make_uint4(pack_half2(v[0], v[1]), pack_half2(v[2], v[3]), pack_half2(v[4], v[5]),
-                    pack_half2(v[6], v[7]));
+  return make_uint4(h[0], h[1], h[2], h[3]);
 }
 
 // Where phase B writes: a flat destination (token t's row at row0 + t * HD)
@@ -417,20 +424,22 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
     if (!ok[t0]) continue;
     const int c0 = 8 * b;      // column in the slice's code rows
     const int cz = cbase + c0;  // channel in the head
-    float a[8], v[8];
+    float2 a[4], v[4];
     {
       const float4 z0 = *reinterpret_cast<const float4*>(zh + cz);
       const float4 z1 = *reinterpret_cast<const float4*>(zh + cz + 4);
       const float4 s0 = *reinterpret_cast<const float4*>(zh + D + cz);
       const float4 s1 = *reinterpret_cast<const float4*>(zh + D + cz + 4);
-      const float z[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-      const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+      const float2 z[4] = {make_float2(z0.x, z0.y), make_float2(z0.z, z0.w),
+                           make_float2(z1.x, z1.y), make_float2(z1.z, z1.w)};
+      const float2 sc[4] = {make_float2(s0.x, s0.y), make_float2(s0.z, s0.w),
+                            make_float2(s1.x, s1.y), make_float2(s1.z, s1.w)};
       const uint2 c = *reinterpret_cast<const uint2*>(codes + t0 * cstride + c0);
       const uint4 hv = dequant8<false>(c, z, sc, a);
       uint16_t* r = row_of<PAGED>(rm, t0);
       if (!PAGED || r) *reinterpret_cast<uint4*>(r + h * D + cz) = hv;
     }
-    const float st[1] = {step};
+    const float2 st[1] = {make_float2(step, step)};
     const int tend = min(kGroup, ntok - t0);
     const uint8_t* cr = codes + t0 * cstride + c0;
     if (gok[g]) {
@@ -450,7 +459,7 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
         }
         if (ADJ) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) a[k] = v[k];
+          for (int k = 0; k < 4; ++k) a[k] = v[k];
         }
       }
     } else {
@@ -465,7 +474,7 @@ __device__ __forceinline__ void dequant_head(const uint8_t* __restrict__ codes, 
         if (!PAGED || row) *reinterpret_cast<uint4*>(row + h * D + cz) = hv;
         if (ADJ) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) a[k] = v[k];
+          for (int k = 0; k < 4; ++k) a[k] = v[k];
         }
       }
     }
