@@ -35,15 +35,15 @@ METRIC = "cg_decode / cg_encode GB/s (fp16 KV) on 1 B200, % of HBM roofline, com
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) per fp16 value of decode_kernel from one ncu capture
 # of the current kernel on a Llama-2-7B-shaped case (32x2x3072x32x128 =
-# 805,306,368 values: 342.2 MB read + 1,552.9 MB written); the bench reports it
+# 805,306,368 values: 352.9 MB read + 1,557.3 MB written); the bench reports it
 # scaled by its own value count.  The capture ends with up to one L2 (126 MB)
 # of written lines not yet in DRAM, so this slightly undercounts.
-DECODE_DRAM_BYTES_PER_VALUE = (342_183_680 + 1_552_913_000) / 805_306_368
+DECODE_DRAM_BYTES_PER_VALUE = (352_920_064 + 1_557_323_000) / 805_306_368
 # Shared-memory wavefronts per warp-symbol of decode_kernel from the same
-# capture (181,248,933 wavefronts for 805,306,368 symbols): the random slot-table
+# capture (189,563,275 wavefronts for 805,306,368 symbols): the random slot-table
 # lookups of 32 streams cost about four, the word refills, the code stores and
 # loads and the table fills the rest.  An SM serves one wavefront per clock.
-DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL = 181_248_933 / (805_306_368 / 32)
+DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL = 189_563_275 / (805_306_368 / 32)
 
 
 def smem_ceiling(symbols: int, ms: float, sm_mhz, sms: int):

@@ -64,11 +64,11 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
 
 
 def test_smem_ceiling_arithmetic():
-    # 32 x 10^9 symbols in 1 s at ~7.2 wavefronts per warp-symbol on 148 SMs at
-    # 1965 MHz: ~7.2e9 wavefronts/s against 290.8e9
+    # 32 x 10^9 symbols in 1 s at ~7.5 wavefronts per warp-symbol on 148 SMs at
+    # 1965 MHz: ~7.5e9 wavefronts/s against 290.8e9
     got = bench.smem_ceiling(32_000_000_000, 1000.0, 1965.0, 148)
     wf = bench.DECODE_SMEM_WAVEFRONTS_PER_WARP_SYMBOL
-    assert 7.1 < wf < 7.3
+    assert 7.4 < wf < 7.6
     assert got["bound"] == "smem" and got["peak"] == round(148 * 1965e6 / 1e9, 1)
     assert abs(got["achieved"] - wf) < 0.06
     assert abs(got["frac"] - wf / 290.82) < 1e-3
