@@ -365,7 +365,10 @@ def run_ours(args):
                          "traffic_source": "ncu dram bytes per value of a 3,072-token "
                                            "Llama-2-7B-shaped capture, scaled by values",
                          "algorithmic_bytes": alg},
-            "gpu_launches": 5 * args.steps,
+            # per step: quant, rans, offsets and compact for each half of the
+            # chunks (cg_encode runs a call of two or more chunks as two
+            # halves on two streams), then one decode
+            "gpu_launches": ((8 if nch >= 2 else 4) + 1) * args.steps,
             "clocks": clocks,
         }
         # what bounds the decode kernel instead of HBM: its shared-memory wavefronts

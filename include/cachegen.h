@@ -85,9 +85,18 @@
  *
  * Conventions of every call below:
  *   - Pointers named *_dev are device memory; everything else is host memory.
- *     The caller owns and allocates every buffer; no call allocates, frees or
- *     synchronises.  All device work is enqueued on `stream` (0 = legacy
- *     default stream) and returns before it completes.
+ *     The caller owns and allocates every buffer; no call allocates device
+ *     memory, frees or synchronises.  All device work is ordered on `stream`
+ *     (0 = legacy default stream) and the calls return before it completes.
+ *     cg_encode and cg_encode_adjacent run the second half of a call of two
+ *     or more chunks on a library-owned stream, forked from `stream` by an
+ *     event before it and joined back into `stream` after it, so work queued
+ *     on `stream` later still sees the whole call done (under graph capture
+ *     the pair is captured as a fork and a join).  That stream and its two
+ *     events are created on the first such call per device and context; a
+ *     call made while `stream` is being captured before they exist runs on
+ *     `stream` alone.  Calls on different streams share the library stream,
+ *     so their second halves run one after the other.
  *   - fp16 values are passed as their uint16_t bit patterns.
  *   - Argument, shape and size errors are returned synchronously and nothing
  *     is enqueued.  Data-dependent errors (corrupt container, non-finite

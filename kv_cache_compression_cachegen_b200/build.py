@@ -25,7 +25,8 @@ NVCC_FLAGS = ARCH + [
     "-Xcompiler", "-fPIC,-O2", "-shared",
 ]
 
-CODEC_SOURCES = ["csrc/capi.cu", "csrc/encode.cu", "csrc/decode.cu", "csrc/static_ws.cu"]
+CODEC_SOURCES = ["csrc/capi.cu", "csrc/encode.cu", "csrc/decode.cu", "csrc/static_ws.cu",
+                 "csrc/context.cu"]
 CODEC_HEADERS = ["csrc/cg_common.cuh"]
 SYNTH_SOURCES = ["synth/kvsynth.cu"]
 

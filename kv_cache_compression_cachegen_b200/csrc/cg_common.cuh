@@ -6,6 +6,7 @@
 #pragma once
 
 #include <cstdint>
+#include <functional>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -240,6 +241,18 @@ struct DecParams {
   int units_per_slab;      // CTAs per (chunk, l, kv)
   int32_t* status;
 };
+
+// Id of the calling thread's current CUDA context; false when there is none
+// (context.cu).
+bool current_context_id(unsigned long long* id);
+
+// Run first(stream) and second(side) with the device's side stream forked from
+// `stream` before them and joined back into it after them (context.cu).  When
+// no side stream can be had (no current context, resources not yet created
+// during a graph capture, creation failed) nothing is queued, *forked stays
+// false and the caller runs its work on `stream` alone.
+cudaError_t fork_join(cudaStream_t stream, const std::function<cudaError_t(cudaStream_t)>& first,
+                      const std::function<cudaError_t(cudaStream_t)>& second, bool* forked);
 
 // Kernel launchers (encode.cu, decode.cu).
 cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stream);

@@ -880,6 +880,44 @@ cudaError_t launch_streams(const EncParams& p, bool check_f, cudaStream_t stream
 
 }  // namespace
 
+namespace {
+
+// Chunks k0, k0 + 1, ... of a call as a call of their own: the containers,
+// their sizes, the supplied tables and every workspace section are laid out
+// chunk by chunk.
+EncParams chunk_tail(const EncParams& p, int k0) {
+  EncParams q = p;
+  const uint64_t k = uint64_t(k0);
+  const uint64_t slabs = uint64_t(p.L) * 2;
+  q.token_start = p.token_start + int64_t(k) * p.C;
+  q.num_chunks = p.num_chunks - k0;
+  q.out = p.out + k * p.out_stride;
+  q.out_sizes = p.out_sizes + k;
+  if (p.tables_in) q.tables_in = p.tables_in + k * p.tables_stride;
+  q.sym = p.sym + k * slabs * p.H * p.D * p.C;
+  q.etab = p.etab + k * slabs * p.H * 256 * 4;
+  q.lens = p.lens + k * slabs * p.C;
+  q.slabtot = p.slabtot + k * slabs;
+  q.scratch = p.scratch + k * slabs * p.C * scratch_stride(p.H, p.D);
+  return q;
+}
+
+cudaError_t launch_encode_one(const EncParams& p, int mode, cudaStream_t stream) {
+  const QSmem sm = q_smem<1>();
+  auto* kern = p.adjacent ? quant_kernel<1, true> : quant_kernel<1, false>;
+  const uint64_t qblocks = uint64_t(p.num_chunks) * p.L * 2 * p.H;
+  kern<<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, mode);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess || mode == kModeTablesOnly) return err;
+  return launch_streams(p, mode == kModeSuppliedTables, stream);
+}
+
+}  // namespace
+
+// A call of two or more chunks runs as two halves, the second on the side
+// stream (fork_join): the halves' kernels overlap, which hides most of one
+// half's memory-bound compaction and loads behind the other's issue-bound
+// rANS encoding.  Without a side stream the call runs on `stream` alone.
 cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stream) {
   const int mode =
       build_only ? kModeTablesOnly : (p.tables_in ? kModeSuppliedTables : kModeEncode);
@@ -888,10 +926,18 @@ cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stre
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm.total));
   if (err != cudaSuccess) return err;
-  const uint64_t qblocks = uint64_t(p.num_chunks) * p.L * 2 * p.H;
-  kern<<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, mode);
-  if ((err = cudaGetLastError()) != cudaSuccess || build_only) return err;
-  return launch_streams(p, mode == kModeSuppliedTables, stream);
+  if (!build_only && p.num_chunks >= 2) {
+    const int half = (p.num_chunks + 1) / 2;
+    EncParams a = p;
+    a.num_chunks = half;
+    const EncParams b = chunk_tail(p, half);
+    bool forked = false;
+    err = fork_join(
+        stream, [&](cudaStream_t s) { return launch_encode_one(a, mode, s); },
+        [&](cudaStream_t s) { return launch_encode_one(b, mode, s); }, &forked);
+    if (forked || err != cudaSuccess) return err;
+  }
+  return launch_encode_one(p, mode, stream);
 }
 
 // Three levels from one quantiser pass: quant_kernel<3> writes every level's

@@ -9,8 +9,6 @@
 // synchronisation of an allocation.  For them this file keeps one fixed block
 // of scratch in device memory, reserved when the library's module is loaded
 // and held by every GPU that loads the library until the process exits.
-#include <cuda.h>  // CUcontext and CUresult types only; the driver calls are looked up at run time
-
 #include <cstdint>
 #include <mutex>
 
@@ -31,39 +29,13 @@ std::mutex g_mutex;
 // The block's device address belongs to the context the module was loaded
 // into.  A device reset destroys that context; the next one loads the module
 // again, possibly elsewhere.  So the cached address is kept together with the
-// unique id of its context (cuCtxGetId) and looked up again when the current
-// context of the device is another one.
+// unique id of its context and looked up again when the current context of
+// the device is another one.
 struct Cached {
   unsigned long long ctx_id;
   void* ptr;
 };
 Cached g_cached[kMaxDevices] = {};
-
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
-CtxGetCurrentFn g_ctx_get_current = nullptr;
-CtxGetIdFn g_ctx_get_id = nullptr;
-
-// Id of the calling thread's current context; false when there is none (or
-// the driver does not offer the calls).  Called with g_mutex held.
-bool current_context_id(unsigned long long* id) {
-  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) {
-    cudaDriverEntryPointQueryResult q1, q2;
-    void* f1 = nullptr;
-    void* f2 = nullptr;
-    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 12000, cudaEnableDefault, &q1) !=
-            cudaSuccess ||
-        cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &q2) !=
-            cudaSuccess ||
-        q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess)
-      return false;
-    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
-    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
-  }
-  CUcontext ctx = nullptr;
-  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
-  return g_ctx_get_id(ctx, id) == CUDA_SUCCESS;
-}
 
 // The array's name is only a host-side handle; the kernels need its device
 // address, looked up with the device current, once per device and context.
@@ -74,14 +46,14 @@ cudaError_t static_workspace(void** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mutex);
   unsigned long long id = 0;
-  if (current_context_id(&id) && g_cached[dev].ptr != nullptr && g_cached[dev].ctx_id == id) {
+  if (cg::current_context_id(&id) && g_cached[dev].ptr != nullptr && g_cached[dev].ctx_id == id) {
     *out = g_cached[dev].ptr;
     return cudaSuccess;
   }
   void* ptr = nullptr;
   err = cudaGetSymbolAddress(&ptr, g_static_workspace);  // also makes the context current
   if (err != cudaSuccess) return err;
-  if (!current_context_id(&id)) return cudaErrorDeviceUninitialized;
+  if (!cg::current_context_id(&id)) return cudaErrorDeviceUninitialized;
   g_cached[dev] = Cached{id, ptr};
   *out = ptr;
   return cudaSuccess;
