@@ -891,14 +891,22 @@ EncParams chunk_tail(const EncParams& p, int k0) {
   const uint64_t slabs = uint64_t(p.L) * 2;
   q.token_start = p.token_start + int64_t(k) * p.C;
   q.num_chunks = p.num_chunks - k0;
-  q.out = p.out + k * p.out_stride;
-  q.out_sizes = p.out_sizes + k;
+  const uint64_t sym_per_chunk = slabs * p.H * p.D * p.C;
+  const uint64_t etab_per_chunk = slabs * p.H * 256 * 4;
+  if (p.out) q.out = p.out + k * p.out_stride;
+  if (p.out_sizes) q.out_sizes = p.out_sizes + k;
   if (p.tables_in) q.tables_in = p.tables_in + k * p.tables_stride;
-  q.sym = p.sym + k * slabs * p.H * p.D * p.C;
-  q.etab = p.etab + k * slabs * p.H * 256 * 4;
+  if (p.sym) q.sym = p.sym + k * sym_per_chunk;
+  if (p.etab) q.etab = p.etab + k * etab_per_chunk;
+  if (p.slabtot) q.slabtot = p.slabtot + k * slabs;
   q.lens = p.lens + k * slabs * p.C;
-  q.slabtot = p.slabtot + k * slabs;
   q.scratch = p.scratch + k * slabs * p.C * scratch_stride(p.H, p.D);
+  for (int j = 0; j < 3; ++j) {  // the three-level encoder's per-level sections
+    if (p.lsym[j]) q.lsym[j] = p.lsym[j] + k * sym_per_chunk;
+    if (p.letab[j]) q.letab[j] = p.letab[j] + k * etab_per_chunk;
+    if (p.lslabtot[j]) q.lslabtot[j] = p.lslabtot[j] + k * slabs;
+    if (p.lout[j]) q.lout[j] = p.lout[j] + k * p.out_stride;
+  }
   return q;
 }
 
@@ -940,18 +948,17 @@ cudaError_t launch_encode(const EncParams& p, bool build_only, cudaStream_t stre
   return launch_encode_one(p, mode, stream);
 }
 
-// Three levels from one quantiser pass: quant_kernel<3> writes every level's
-// symbols, tables and encoder constants; then each level's streams are encoded
-// and compacted in turn (the stream lengths and word slots are reused).
-cudaError_t launch_encode_levels(const EncParams& p, uint64_t* out_sizes, cudaStream_t stream) {
+namespace {
+
+// Chunks of a three-level call (p already covers them; k0 is the first one's
+// index in the call, whose container sizes are laid out [level][chunk]).
+cudaError_t launch_levels_part(const EncParams& p, uint64_t* out_sizes, int total_chunks, int k0,
+                               cudaStream_t stream) {
   const QSmem sm = q_smem<3>();
-  cudaError_t err = cudaFuncSetAttribute(quant_kernel<3, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(sm.total));
-  if (err != cudaSuccess) return err;
   const uint64_t qblocks = uint64_t(p.num_chunks) * p.L * 2 * p.H;
   quant_kernel<3, false><<<unsigned(qblocks), kQThreads, sm.total, stream>>>(p, kModeEncode);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
   for (int j = 0; j < 3; ++j) {
     EncParams q = p;
     q.level = j;
@@ -959,10 +966,38 @@ cudaError_t launch_encode_levels(const EncParams& p, uint64_t* out_sizes, cudaSt
     q.etab = p.letab[j];
     q.slabtot = p.lslabtot[j];
     q.out = p.lout[j];
-    q.out_sizes = out_sizes + uint64_t(j) * p.num_chunks;
+    q.out_sizes = out_sizes + uint64_t(j) * total_chunks + k0;
     if ((err = launch_streams(q, false, stream)) != cudaSuccess) return err;
   }
   return cudaSuccess;
+}
+
+}  // namespace
+
+// Three levels from one quantiser pass: quant_kernel<3> writes every level's
+// symbols, tables and encoder constants; then each level's streams are encoded
+// and compacted in turn (the stream lengths and word slots are reused).  As in
+// launch_encode, a call of two or more chunks runs as two halves on two
+// streams.
+cudaError_t launch_encode_levels(const EncParams& p, uint64_t* out_sizes, cudaStream_t stream) {
+  const QSmem sm = q_smem<3>();
+  cudaError_t err = cudaFuncSetAttribute(quant_kernel<3, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(sm.total));
+  if (err != cudaSuccess) return err;
+  const int n = p.num_chunks;
+  if (n >= 2) {
+    const int half = (n + 1) / 2;
+    EncParams a = p;
+    a.num_chunks = half;
+    const EncParams b = chunk_tail(p, half);
+    bool forked = false;
+    err = fork_join(
+        stream, [&](cudaStream_t s) { return launch_levels_part(a, out_sizes, n, 0, s); },
+        [&](cudaStream_t s) { return launch_levels_part(b, out_sizes, n, half, s); }, &forked);
+    if (forked || err != cudaSuccess) return err;
+  }
+  return launch_levels_part(p, out_sizes, n, 0, stream);
 }
 
 }  // namespace cg
