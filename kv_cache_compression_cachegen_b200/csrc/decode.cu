@@ -11,26 +11,29 @@
 // CTA = one "unit": 32 anchor groups (320 tokens) of one (chunk, layer, K/V);
 // thread t decodes the stream of local token t (anchors and deltas alike).
 // Every stream holds H*D symbols in [h][d] order and every head has its own
-// frequency table, so the CTA walks the heads in lockstep, two phases per head:
+// frequency table, so the CTA walks the heads in lockstep.  Each head is
+// taken in two slices of D/2 channels, two phases per slice:
 //
-//   phase A  every thread decodes the D symbols of head h of its stream and
+//   phase A  every thread decodes the slice's D/2 symbols of its stream and
 //            leaves the byte codes u = q + 127 in shared memory, codes[t][d];
 //            the only shared-memory traffic is the slot-table lookup, the word
 //            refill and one 8-byte code store per 8 symbols.
-//   phase B  the threads turn the codes of head h into fp16.  A work item is
+//   phase B  the threads turn the slice's codes into fp16.  A work item is
 //            (anchor group g, 8 channels): the anchor's values
 //            a = zp + (float)c * scale, then the nine deltas a + (float)q * step
 //            (format 2: each delta against the previous token's value), all
 //            fp32 with IEEE round-to-nearest adds and multiplies (no
 //            contraction), each row's 8 values leaving as one 16-byte store;
 //            consecutive lanes take consecutive channel blocks, so a warp's
-//            stores cover whole row segments.  Meanwhile the slot table is
-//            rebuilt for head h + 1 (phase A of head h no longer reads it) and
-//            the zero points / scales of head h + 1 are staged.
+//            stores cover whole row segments.  After the head's last slice the
+//            slot table is rebuilt for head h + 1 (phase A of head h no longer
+//            reads it) and the zero points / scales of head h + 1 are staged.
 //
-// A __syncthreads separates the phases (two per head).  Anchors get no special treatment in
-// phase A, and the reconstructed anchors never leave the registers of the
-// phase-B item, so the work of a head is spread evenly over the CTA.
+// A __syncthreads separates the phases (four per head).  Anchors get no
+// special treatment in phase A, and the reconstructed anchors never leave the
+// registers of the phase-B item, so the work of a head is spread evenly over
+// the CTA.  Half a head of codes keeps a CTA at about 72 KB of shared memory,
+// so three CTAs (30 warps) share an SM.
 //
 // Compressed words reach a thread through a 64-byte ring in shared memory
 // (four 16-byte blocks, plus a copy of the first block after the last, so that
