@@ -25,6 +25,9 @@
 //                   scan of its stream lengths -> offsets; the last one of a
 //                   chunk writes the header and the container size.
 //   compact_kernel  one warp per stream: scratch slot -> payload.
+//
+// A call of two or more chunks runs this sequence twice, once per half of its
+// chunks, the second half on the library's side stream (launch_encode).
 #include <cuda_fp16.h>
 
 #include "cg_common.cuh"
