@@ -300,6 +300,18 @@ cg_status cg_decode_adjacent_into(const cg_shape* shape, const uint8_t* in_dev,
                                   cg_level level, uint16_t* kv_dev, int64_t total_tokens,
                                   int32_t* status_dev, cudaStream_t stream);
 
+/* cg_decode_into_paged of format-2 containers (same arguments and pool
+ * layout).  A token whose page is unmapped is not written and sets
+ * CG_ERR_MISMATCH; the later tokens of its group are still written, because
+ * each group's chain is rebuilt from the decoded values, never read back from
+ * the pool. */
+cg_status cg_decode_adjacent_into_paged(const cg_shape* shape, const uint8_t* in_dev,
+                                        uint64_t in_stride, int32_t num_chunks,
+                                        int32_t chunk_tokens, cg_level level, uint16_t* pool_dev,
+                                        int32_t num_pages, int32_t page_tokens,
+                                        const int32_t* block_table_dev, int64_t total_tokens,
+                                        int32_t* status_dev, cudaStream_t stream);
+
 /* Device workspace cg_encode_levels needs for `num_chunks` chunks of
  * `chunk_tokens` (about three times the symbol part of cg_encode's).  Host,
  * pure. */

@@ -19,7 +19,7 @@ __all__ = [
     "Shape", "library", "library_path", "check", "cg_status_string", "cg_section_offsets",
     "cg_encoded_bound", "cg_tables_bytes", "cg_encode_workspace_bytes", "cg_build_tables",
     "cg_encode", "cg_encode_static", "cg_encode_levels", "cg_encode_levels_workspace_bytes",
-    "cg_encode_adjacent", "cg_decode_adjacent", "cg_decode_adjacent_into", "cg_decode", "cg_decode_into", "cg_decode_into_paged",
+    "cg_encode_adjacent", "cg_decode_adjacent", "cg_decode_adjacent_into", "cg_decode_adjacent_into_paged", "cg_decode", "cg_decode_into", "cg_decode_into_paged",
 ]
 
 CG_OK, CG_ERR_INVALID_ARG, CG_ERR_CAPACITY, CG_ERR_CORRUPT = 0, 1, 2, 3
@@ -97,6 +97,10 @@ _SIGNATURES = {
                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_int, _P,
                                             ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int64,
                                             _P, _P]),
+    "cg_decode_adjacent_into_paged": (ctypes.c_int, [ctypes.POINTER(Shape), _P, ctypes.c_uint64,
+                                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_int,
+                                                     _P, ctypes.c_int32, ctypes.c_int32, _P,
+                                                     ctypes.c_int64, _P, _P]),
 }
 
 _lib = None
@@ -266,3 +270,13 @@ def cg_decode_into_paged(shape, inp, in_stride: int, num_chunks: int, chunk_toke
                                           num_chunks, chunk_tokens, int(level), _ptr(pool),
                                           num_pages, page_tokens, _ptr(block_table),
                                           total_tokens, _ptr(status), _stream(stream))
+
+
+def cg_decode_adjacent_into_paged(shape, inp, in_stride: int, num_chunks: int,
+                                  chunk_tokens: int, level: int, pool, num_pages: int,
+                                  page_tokens: int, block_table, total_tokens: int, status,
+                                  stream=None) -> int:
+    return library().cg_decode_adjacent_into_paged(
+        ctypes.byref(_shape(shape)), _ptr(inp), in_stride, num_chunks, chunk_tokens, int(level),
+        _ptr(pool), num_pages, page_tokens, _ptr(block_table), total_tokens, _ptr(status),
+        _stream(stream))

@@ -385,4 +385,22 @@ cg_status cg_decode_into_paged(const cg_shape* shape, const uint8_t* in_dev, uin
                        page_tokens);
 }
 
+cg_status cg_decode_adjacent_into_paged(const cg_shape* shape, const uint8_t* in_dev,
+                                        uint64_t in_stride, int32_t num_chunks,
+                                        int32_t chunk_tokens, cg_level level, uint16_t* pool_dev,
+                                        int32_t num_pages, int32_t page_tokens,
+                                        const int32_t* block_table_dev, int64_t total_tokens,
+                                        int32_t* status_dev, cudaStream_t stream) {
+  cg_status st = check_decode_args(shape, in_dev, in_stride, num_chunks, chunk_tokens, level,
+                                   pool_dev, status_dev);
+  if (st != CG_OK) return st;
+  if (total_tokens < 1 || num_pages < 1 || page_tokens < 1 || block_table_dev == nullptr)
+    return CG_ERR_INVALID_ARG;
+  const uint64_t elems = uint64_t(shape->num_layers) * 2 * uint64_t(num_pages) *
+                         uint64_t(page_tokens) * shape->num_kv_heads * shape->head_dim;
+  return decode_common(shape, in_dev, in_stride, num_chunks, chunk_tokens, level, pool_dev,
+                       elems, 2, total_tokens, status_dev, stream, block_table_dev, num_pages,
+                       page_tokens, 1);
+}
+
 }  // extern "C"

@@ -13,8 +13,8 @@ from dataclasses import dataclass
 import torch
 
 from . import (CG_OK, CacheGenError, Shape, cg_build_tables, cg_decode, cg_decode_adjacent,
-               cg_decode_adjacent_into, cg_decode_into, cg_decode_into_paged, cg_encode,
-               cg_encode_adjacent, cg_encode_levels,
+               cg_decode_adjacent_into, cg_decode_adjacent_into_paged, cg_decode_into,
+               cg_decode_into_paged, cg_encode, cg_encode_adjacent, cg_encode_levels,
                cg_encode_levels_workspace_bytes, cg_encode_workspace_bytes, cg_encoded_bound,
                cg_tables_bytes, check)
 
@@ -179,16 +179,17 @@ def decode_into(data: torch.Tensor, stride: int, shape: Shape, chunk_tokens: int
 def decode_into_paged(data: torch.Tensor, stride: int, shape: Shape, chunk_tokens: int,
                       level: int, num_chunks: int, pool: torch.Tensor, page_tokens: int,
                       block_table: torch.Tensor, total_tokens: int,
-                      status: torch.Tensor | None = None, stream=None):
+                      status: torch.Tensor | None = None, stream=None, adjacent: bool = False):
     """Decode into a paged pool [L][2][num_pages][page_tokens][H][D] through an
-    int32 block table (logical page -> physical page)."""
+    int32 block table (logical page -> physical page).  adjacent=True decodes
+    format-2 containers."""
     L, H, D = shape.num_layers, shape.num_kv_heads, shape.head_dim
     num_pages = pool.numel() // (L * 2 * page_tokens * H * D)
     if status is None:
         status = new_status(data.device)
-    check(cg_decode_into_paged(shape, data, stride, num_chunks, chunk_tokens, level, pool,
-                               num_pages, page_tokens, block_table, total_tokens, status,
-                               stream), "cg_decode_into_paged")
+    fn = cg_decode_adjacent_into_paged if adjacent else cg_decode_into_paged
+    check(fn(shape, data, stride, num_chunks, chunk_tokens, level, pool, num_pages, page_tokens,
+             block_table, total_tokens, status, stream), fn.__name__)
     return status
 
 

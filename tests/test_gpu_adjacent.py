@@ -189,3 +189,52 @@ def test_corrupt_format2_containers_report_a_status():
     buf[secs[4] + 100] ^= 0x10
     assert status(buf, enc.stride) == oracle.CORRUPT
     assert status(torch.zeros_like(enc.data), enc.stride, into=True) == oracle.CORRUPT
+
+
+def test_format2_into_paged_pool():
+    # Format-2 containers decoded into a paged pool through a shuffled block
+    # table: every logical token's row equals the oracle's format-2 decode.
+    L, H, D, T, C, P = 3, 2, 64, 250, 96, 16
+    kv = gu.gen(L, H, D, T, seed=21)
+    shape = Shape(L, H, D)
+    nch = -(-T // C)
+    enc = ta.encode(kv, C, 1, adjacent=True)
+    torch.cuda.synchronize()
+    assert ta.status_of(enc.status) == 0
+    npages_logical = -(-T // P)
+    num_pages = npages_logical + 3
+    g = torch.Generator().manual_seed(5)
+    table = torch.randperm(num_pages, generator=g)[:npages_logical].to(torch.int32).cuda()
+    pool = torch.full((L, 2, num_pages, P, H, D), 0x7E00, dtype=torch.int16, device="cuda")
+    st = ta.decode_into_paged(enc.data, enc.stride, shape, C, 1, nch, pool, P, table, T,
+                              adjacent=True)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == 0
+    conts = gu.gpu_containers(enc, range(nch))
+    dref = _oracle_v2_decodes(conts, shape, C, 1)
+    logical = gu.host(pool[:, :, table.long()].reshape(L, 2, npages_logical * P, H, D))
+    for k in range(nch):
+        n = min(C, T - k * C)
+        assert np.array_equal(logical[:, :, k * C:k * C + n], dref[k]), k
+    tab = table.cpu().tolist()
+    unused = sorted(set(range(num_pages)) - set(tab))
+    assert bool((pool[:, :, unused] == 0x7E00).all())
+
+    # Logical page 3 (tokens 48..63) unmapped: its rows are not written, the
+    # call reports a mismatch, and the later tokens of the groups it cuts
+    # (the group of tokens 60..69 continues on page 4) still decode exactly.
+    bad = table.clone()
+    bad[3] = num_pages
+    pool2 = torch.full_like(pool, 0x7E00)
+    st = ta.decode_into_paged(enc.data, enc.stride, shape, C, 1, nch, pool2, P, bad, T,
+                              adjacent=True)
+    torch.cuda.synchronize()
+    assert ta.status_of(st) == CG_ERR_MISMATCH
+    badtab = bad.cpu().tolist()
+    for lp in range(npages_logical):
+        a, b = lp * P, min(T, (lp + 1) * P)
+        if lp == 3:
+            continue
+        assert torch.equal(pool2[:, :, badtab[lp], :b - a], pool[:, :, tab[lp], :b - a]), lp
+    # the physical page logical page 3 used to map to was never written
+    assert bool((pool2[:, :, tab[3]] == 0x7E00).all())
