@@ -355,6 +355,36 @@ __device__ __forceinline__ void decode_codes(uint32_t& x, uint32_t& p, uint32_t&
   }
 }
 
+// Packed fp32 pair arithmetic (sm_100 f32x2): each component rounds like the
+// scalar instruction with the same modifier.  A packed multiply feeding a
+// packed add did not give RN(a + RN(q * s)) on sm_100a (most cancelling sums
+// differed, as from a fused multiply-add), even with the rounding modifier
+// written out, so a product is only ever added with the scalar __fadd_rn,
+// which is never contracted.
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // (float)(u - 127) for bytes K and K + 1 of a word of codes: the bits
 // 0x4B0000uu are the float 2^23 + u, and subtracting 2^23 + 127 is exact.
 template <int K>
