@@ -129,3 +129,43 @@ def test_graph_capture_before_the_side_stream_exists():
                          text=True, timeout=600, env=env)
     assert res.returncode == 0, res.stdout[-2000:] + res.stderr[-4000:]
     assert "fresh-capture-ok" in res.stdout
+
+
+def test_concurrent_calls_from_two_host_threads():
+    # The side stream and its fork/join events are shared by every call on the
+    # device: calls from two host threads on two streams must still produce
+    # their own bytes (ctypes releases the GIL inside the C call).
+    import threading
+    L, H, D, C = 4, 4, 64, 256
+    T = 3 * C + 40
+    kvs = [gu.gen(L, H, D, T, seed=30 + i) for i in range(2)]
+    shape = Shape(L, H, D)
+    refs = []
+    for kv in kvs:
+        refs.append(_containers(ta.encode(kv, C, 1)))
+        torch.cuda.synchronize()
+    encs = [ta.Encoder(shape, C, -(-T // C), kvs[0].device) for _ in range(2)]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    errors = []
+
+    def worker(i):
+        try:
+            with torch.cuda.stream(streams[i]):
+                for _ in range(20):
+                    encs[i].encode(kvs[i], 1, stream=streams[i])
+            streams[i].synchronize()
+        except Exception as e:  # reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    torch.cuda.synchronize()
+    for i in range(2):
+        assert ta.status_of(encs[i].status) == 0
+        got = _containers(ta.Encoded(encs[i].out, encs[i].sizes, encs[i].stride,
+                                     encs[i].num_chunks, C, 1, shape, encs[i].status))
+        assert all(np.array_equal(a, b) for a, b in zip(got, refs[i])), i
